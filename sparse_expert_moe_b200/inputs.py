@@ -1,0 +1,313 @@
+"""Seeded synthetic inputs for the MoE layer.
+
+This module is shared by the oracle tests, the GPU parity tests, ``bench.py``
+and ``smoke()``.  It holds none of the layer's arithmetic: it only draws
+random numbers, encodes the drawn values in the storage types the layer
+consumes (bf16 round-to-nearest-even, e4m3 with power-of-two block scales),
+and applies a stored per-workload recipe (rows to redraw so that routing has a
+score margin, and for the Zipf workloads a fitted selection bias).  Recipes are
+JSON files under ``tests/golden/recipes/``, written by
+``tests/golden/make_recipes.py``, which computes them with the oracle only.
+
+Every tensor is drawn from its own numpy ``Generator(PCG64)`` stream keyed by
+(seed, family, tensor, index), so one expert's weights can be redrawn alone
+and the result does not depend on the number of threads used.
+
+Workloads (shapes from the pages: DeepSeek R1 in the InferenceX v2 claim
+record IX2-0397, section "WideEP" -- 256 routed experts, 1 shared, 8 per
+token; "Decoding Trillion-Parameter MoE LLMs", section "Expert Granularity:
+More, Smaller Experts" -- 384 experts, top-8 plus one shared expert):
+
+  tiny            T=64   d=128  E=8   k=2 I=256  S=0 softmax       fp32
+  r1_decode       T=128  d=7168 E=256 k=8 I=2048 S=1 sigmoid+bias  bf16
+  r1_prefill      T=8192 d=7168 E=256 k=8 I=2048 S=1 sigmoid+bias  bf16, Zipf(1.1) loads
+  kimi            T=4096 d=7168 E=384 k=8 I=2048 S=1 sigmoid+bias  bf16
+  r1_prefill_fp8  r1_prefill with e4m3 activations (1x128 scales) and e4m3
+                  weights (128x128 scales), bf16 output
+"""
+from __future__ import annotations
+
+import json
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field, replace
+from typing import Optional
+
+import numpy as np
+import torch
+
+RECIPE_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                          "tests", "golden", "recipes")
+
+# stream ids
+_X, _WR, _BIAS, _W13, _W2, _WS13, _WS2, _XRE, _LOGITS, _ZIPF = range(1, 11)
+_FAMILY = {"tiny": 1, "r1": 2, "kimi": 3, "custom": 9}
+
+W_STD = 0.02
+E4M3_MAX = 448.0
+
+
+@dataclass(frozen=True)
+class Spec:
+    name: str
+    T: int
+    d_model: int
+    E: int
+    top_k: int
+    d_ff: int
+    n_shared: int
+    score: str            # "softmax" | "sigmoid_bias"
+    act: str              # "f32" | "bf16" | "e4m3"
+    weight: str           # "f32" | "bf16" | "e4m3"
+    out: str              # "f32" | "bf16"
+    family: str           # weight-draw family: workloads of one family share weights
+    x_stream: int         # activation-draw stream
+    loads: str = "uniform"            # "uniform" | "zipf"
+    bias_range: Optional[float] = None  # sel bias ~ U(-r, r) when drawn
+    margin: float = 1e-3
+    zipf_s: float = 1.1
+
+
+SPECS = {
+    "tiny": Spec("tiny", 64, 128, 8, 2, 256, 0, "softmax", "f32", "f32", "f32",
+                 family="tiny", x_stream=1, margin=1e-2),
+    "r1_decode": Spec("r1_decode", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "bf16", "bf16",
+                      "bf16", family="r1", x_stream=2, bias_range=0.1),
+    "r1_prefill": Spec("r1_prefill", 8192, 7168, 256, 8, 2048, 1, "sigmoid_bias", "bf16", "bf16",
+                       "bf16", family="r1", x_stream=3, loads="zipf"),
+    "kimi": Spec("kimi", 4096, 7168, 384, 8, 2048, 1, "sigmoid_bias", "bf16", "bf16", "bf16",
+                 family="kimi", x_stream=4),
+    "r1_prefill_fp8": Spec("r1_prefill_fp8", 8192, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
+                           "e4m3", "bf16", family="r1", x_stream=3, loads="zipf"),
+}
+
+# the Zipf workload whose fitted selection bias the FP8 variant reuses
+BIAS_SOURCE = {"r1_prefill_fp8": "r1_prefill"}
+
+
+def custom_spec(T, d_model, E, top_k, d_ff, n_shared=0, score="sigmoid_bias", act="bf16",
+                weight="bf16", out="bf16", bias_range=0.1, x_stream=7, margin=1e-3):
+    """A small workload for parity tests (own weight family, no stored recipe)."""
+    return Spec(f"custom_T{T}_d{d_model}_E{E}_k{top_k}_I{d_ff}_S{n_shared}", T, d_model, E, top_k,
+                d_ff, n_shared, score, act, weight, out, family="custom", x_stream=x_stream,
+                bias_range=bias_range if score == "sigmoid_bias" else None, margin=margin)
+
+
+def _rng(seed, *key):
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), *map(int, key)])))
+
+
+# ---------------------------------------------------------------------------
+# storage encodings of drawn values
+# ---------------------------------------------------------------------------
+
+def to_bf16(a: np.ndarray) -> torch.Tensor:
+    """fp32 draw -> bf16 tensor (round to nearest even)."""
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _pow2_scale(amax: np.ndarray) -> np.ndarray:
+    """Smallest power of two s with amax / s <= 448 (1.0 for an all-zero block)."""
+    v = np.asarray(amax, np.float64) / E4M3_MAX
+    m, e = np.frexp(v)                  # v = m * 2^e, m in [0.5, 1)
+    e = np.where(m == 0.5, e - 1, e)    # exact powers of two
+    s = np.ldexp(1.0, e.astype(np.int64))
+    return np.where(v > 0, s, 1.0).astype(np.float32)
+
+
+def to_e4m3_blocks(a: np.ndarray, br: int, bc: int):
+    """fp32 draw [R, C] -> (e4m3 codes as torch.float8_e4m3fn [R, C], fp32 scales [R/br, C/bc])."""
+    R, C = a.shape
+    blocks = np.abs(a).reshape(R // br, br, C // bc, bc).max(axis=(1, 3))
+    s = _pow2_scale(blocks)
+    full = np.repeat(np.repeat(s, br, axis=0), bc, axis=1)
+    q = torch.from_numpy(np.ascontiguousarray(a / full, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return q, torch.from_numpy(s)
+
+
+# ---------------------------------------------------------------------------
+# draws
+# ---------------------------------------------------------------------------
+
+def _draw_x_fp32(spec: Spec, seed: int, redraw) -> np.ndarray:
+    x = _rng(seed, _FAMILY[spec.family], _X, spec.x_stream).standard_normal(
+        (spec.T, spec.d_model), dtype=np.float32)
+    for t, attempt in (redraw or []):
+        x[t] = redraw_row(spec, seed, t, attempt)
+    return x
+
+
+def redraw_row(spec: Spec, seed: int, t: int, attempt: int) -> np.ndarray:
+    """Replacement draw number ``attempt`` (>= 1) for activation row t."""
+    return _rng(seed, _FAMILY[spec.family], _XRE, spec.x_stream, t, attempt).standard_normal(
+        spec.d_model, dtype=np.float32)
+
+
+def encode_act(spec: Spec, x32: np.ndarray):
+    if spec.act == "f32":
+        return torch.from_numpy(np.ascontiguousarray(x32)), None
+    if spec.act == "bf16":
+        return to_bf16(x32), None
+    if spec.act == "e4m3":
+        return to_e4m3_blocks(x32, 1, 128)
+    raise ValueError(spec.act)
+
+
+def _encode_weight(spec: Spec, w32: np.ndarray):
+    if spec.weight == "f32":
+        return torch.from_numpy(np.ascontiguousarray(w32)), None
+    if spec.weight == "bf16":
+        return to_bf16(w32), None
+    if spec.weight == "e4m3":
+        return to_e4m3_blocks(w32, 128, 128)
+    raise ValueError(spec.weight)
+
+
+def draw_expert(spec: Spec, seed: int, e: int, shared: bool = False):
+    """(w13, w13_scale, w2, w2_scale) of routed expert e or shared expert e."""
+    fam = _FAMILY[spec.family]
+    I, d = spec.d_ff, spec.d_model
+    r13 = _rng(seed, fam, _WS13 if shared else _W13, e)
+    w13 = r13.standard_normal((2 * I, d), dtype=np.float32)
+    w13 *= np.float32(W_STD)
+    r2 = _rng(seed, fam, _WS2 if shared else _W2, e)
+    w2 = r2.standard_normal((d, I), dtype=np.float32)
+    w2 *= np.float32(W_STD)
+    q13, s13 = _encode_weight(spec, w13)
+    q2, s2 = _encode_weight(spec, w2)
+    return q13, s13, q2, s2
+
+
+def draw_router(spec: Spec, seed: int):
+    wr = _rng(seed, _FAMILY[spec.family], _WR, 0).standard_normal((spec.E, spec.d_model),
+                                                                  dtype=np.float32)
+    wr *= np.float32(W_STD)
+    if spec.weight == "f32":
+        return torch.from_numpy(wr)
+    return to_bf16(wr)   # router weights are bf16 for the bf16 and e4m3 workloads
+
+
+def draw_sel_bias(spec: Spec, seed: int):
+    if spec.bias_range is None:
+        return None
+    r = spec.bias_range
+    b = _rng(seed, _FAMILY[spec.family], _BIAS, spec.x_stream).uniform(-r, r, spec.E)
+    return torch.from_numpy(b.astype(np.float32))
+
+
+def zipf_assignment(spec: Spec, seed: int) -> np.ndarray:
+    """Target expert loads: k distinct experts per token drawn by Gumbel-top-k from Zipf(s) weights.
+
+    Rank r (1-based) has weight r^-s; ranks map to expert ids by a seeded permutation.
+    Returns the per-expert target counts [E].
+    """
+    g = _rng(seed, _FAMILY[spec.family], _ZIPF, spec.x_stream)
+    ranks = np.arange(1, spec.E + 1, dtype=np.float64)
+    logw = -spec.zipf_s * np.log(ranks)
+    expert_of_rank = g.permutation(spec.E)
+    gumbel = g.gumbel(size=(spec.T, spec.E))
+    pick = np.argsort(-(logw[None, :] + gumbel), axis=1, kind="stable")[:, : spec.top_k]
+    counts = np.bincount(expert_of_rank[pick].ravel(), minlength=spec.E)
+    return counts
+
+
+def draw_logits(T: int, E: int, seed: int, lo=-3.0, hi=3.0, redraw=None, stream=0):
+    """fp32 router logits U(lo, hi) supplied directly to the routing kernels."""
+    L = _rng(seed, _FAMILY["custom"], _LOGITS, stream, T, E).uniform(lo, hi, (T, E)).astype(np.float32)
+    for t, attempt in (redraw or []):
+        L[t] = _rng(seed, _FAMILY["custom"], _LOGITS, stream, T, E, t, attempt).uniform(
+            lo, hi, E).astype(np.float32)
+    return L
+
+
+# ---------------------------------------------------------------------------
+# whole workloads
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Workload:
+    spec: Spec
+    seed: int
+    x: torch.Tensor                       # [T, d] f32 | bf16 | float8_e4m3fn
+    x_scale: Optional[torch.Tensor]       # [T, d/128] fp32 (e4m3 only)
+    wr: torch.Tensor                      # [E, d]
+    sel_bias: Optional[torch.Tensor]      # [E] fp32
+    w13: torch.Tensor                     # [E, 2I, d]
+    w13_s: Optional[torch.Tensor]         # [E, 2I/128, d/128]
+    w2: torch.Tensor                      # [E, d, I]
+    w2_s: Optional[torch.Tensor]          # [E, d/128, I/128]
+    ws13: Optional[torch.Tensor]          # [S, 2I, d]
+    ws13_s: Optional[torch.Tensor]
+    ws2: Optional[torch.Tensor]           # [S, d, I]
+    ws2_s: Optional[torch.Tensor]
+    recipe: dict = field(default_factory=dict)
+
+
+def _stack_experts(spec, seed, n, shared, threads):
+    I, d = spec.d_ff, spec.d_model
+    wdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[spec.weight]
+    w13 = torch.empty((n, 2 * I, d), dtype=wdt)
+    w2 = torch.empty((n, d, I), dtype=wdt)
+    scaled = spec.weight == "e4m3"
+    s13 = torch.empty((n, 2 * I // 128, d // 128), dtype=torch.float32) if scaled else None
+    s2 = torch.empty((n, d // 128, I // 128), dtype=torch.float32) if scaled else None
+
+    def one(e):
+        q13, a13, q2, a2 = draw_expert(spec, seed, e, shared)
+        w13[e].copy_(q13)
+        w2[e].copy_(q2)
+        if scaled:
+            s13[e].copy_(a13)
+            s2[e].copy_(a2)
+
+    if n:
+        with ThreadPoolExecutor(max(1, min(threads, n))) as ex:
+            list(ex.map(one, range(n)))
+    return w13, s13, w2, s2
+
+
+def load_recipe(name: str) -> dict:
+    path = os.path.join(RECIPE_DIR, f"{name}.json")
+    with open(path) as f:
+        return json.load(f)
+
+
+def make_workload(spec: Spec, seed: int = 0, redraw=None, sel_bias=None, threads=None,
+                  recipe=None) -> Workload:
+    """Draw every input of one layer call."""
+    threads = threads or os.cpu_count() or 1
+    x32 = _draw_x_fp32(spec, seed, redraw)
+    x, x_scale = encode_act(spec, x32)
+    del x32
+    wr = draw_router(spec, seed)
+    if sel_bias is None:
+        sel_bias = draw_sel_bias(spec, seed)
+    elif not isinstance(sel_bias, torch.Tensor):
+        sel_bias = torch.tensor(np.asarray(sel_bias, np.float32))
+    w13, w13_s, w2, w2_s = _stack_experts(spec, seed, spec.E, False, threads)
+    if spec.n_shared:
+        ws13, ws13_s, ws2, ws2_s = _stack_experts(spec, seed, spec.n_shared, True, threads)
+    else:
+        ws13 = ws13_s = ws2 = ws2_s = None
+    return Workload(spec, seed, x, x_scale, wr, sel_bias, w13, w13_s, w2, w2_s,
+                    ws13, ws13_s, ws2, ws2_s, recipe or {})
+
+
+def load_workload(name: str, seed: int = 0, threads=None, T: Optional[int] = None) -> Workload:
+    """A named workload with its stored recipe applied (seed 0 recipes are committed).
+
+    ``T`` may shrink the token count (rows 0..T-1 of the same draw).
+    """
+    spec = SPECS[name]
+    recipe = load_recipe(name) if seed == 0 else {}
+    bias = recipe.get("sel_bias")
+    if bias is None and name in BIAS_SOURCE and seed == 0:
+        bias = load_recipe(BIAS_SOURCE[name]).get("sel_bias")
+    w = make_workload(spec, seed, redraw=recipe.get("redraw"), sel_bias=bias, threads=threads,
+                      recipe=recipe)
+    if T is not None and T != spec.T:
+        w.spec = replace(spec, T=T)
+        w.x = w.x[:T].contiguous()
+        if w.x_scale is not None:
+            w.x_scale = w.x_scale[:T].contiguous()
+    return w
