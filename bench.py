@@ -1,0 +1,476 @@
+"""Throughput of the MoE feed-forward layer on B200: one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload r1_decode] [--impl reference]
+
+A step is one ``moe_layer_forward`` (router GEMM, route, permute, tile plan,
+grouped SwiGLU FFN for routed + shared experts, combine) over one batch of T
+tokens with the weights resident in HBM.  ``value`` is tokens/s over all
+ranks (replicas: the layer does not shard on this path, so each rank runs its
+own copy), timed with CUDA events between a barrier + synchronize on both
+sides, max over ranks.  ``e2e`` is the same metric through the public call with
+the activations copied in from pinned host memory and the output copied back
+every step.  The per-stage times come from ``moe_layer_forward_staged`` events
+recorded inside the timed steps; ``roofline`` is the dominant kernel's
+algorithmic bytes (or flops) per launch over its average in-place duration.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at 1 B200; % of HBM (decode) / tensor (prefill) roofline"
+DEFAULT_WORKLOAD = "r1_decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# kernels this library launches per layer call (bf16 family): router GEMM, route,
+# permute (count/scan, rank, gather), tile plan, FFN1, FFN2, combine
+LAUNCHES_PER_STEP = 9
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, else nvidia-smi)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._dev = device_index
+        self._thread = None
+
+    def _run(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self._dev)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_r = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop.is_set():
+                self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                r = get_r(h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+                time.sleep(0.02)
+            pynvml.nvmlShutdown()
+        except Exception as e:  # NVML missing: one nvidia-smi reading instead
+            self.samples.append(None)
+            self.error = repr(e)
+
+    def __enter__(self):
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._thread.join(timeout=5)
+
+    def summary(self):
+        vals = [s for s in self.samples if s]
+        return {"sm_mhz": statistics.median(vals) if vals else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(vals)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def work_model(spec, offsets):
+    """Algorithmic bytes / flops of the layer and of its two expert GEMM launches.
+
+    Decode units: the weight bytes of every expert that received at least one
+    row (plus the shared experts and the router) -- a dense pass over all
+    experts is not the measure.  Prefill units: 2 * rows * 3 * d * I flops over
+    the routed and shared rows plus the router's 2 * T * d * E.
+    """
+    T, d, E, k, I, S = spec.T, spec.d_model, spec.E, spec.top_k, spec.d_ff, spec.n_shared
+    wb = 1 if spec.weight == "e4m3" else 2
+    ab = 1 if spec.act == "e4m3" else 2
+    sizes = np.diff(offsets)
+    touched = int((sizes > 0).sum())
+    R = T * k
+    rows = R + S * T
+    ffn1_bytes = (touched + S) * 2 * I * d * wb + rows * d * ab + rows * I * 2
+    ffn2_bytes = (touched + S) * d * I * wb + rows * I * 2 + rows * d * 2
+    layer_weight_bytes = (touched + S) * 3 * I * d * wb + E * d * 2
+    ffn1_flops = 2.0 * rows * 2 * I * d
+    ffn2_flops = 2.0 * rows * I * d
+    layer_flops = 2.0 * rows * 3 * I * d + 2.0 * T * d * E
+    return dict(touched=touched, ffn1_bytes=ffn1_bytes, ffn2_bytes=ffn2_bytes,
+                layer_weight_bytes=layer_weight_bytes, ffn1_flops=ffn1_flops,
+                ffn2_flops=ffn2_flops, layer_flops=layer_flops)
+
+
+def bound_of(name):
+    return "tensor" if name in ("r1_prefill", "r1_prefill_fp8") else "hbm"
+
+
+def read_traffic(kernel_key):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = os.path.join(ROOT, "sparse_expert_moe_b200", "csrc", "grouped_gemm.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for ln in lines:
+        parts = ln.split()
+        if len(parts) >= 3 and parts[0] == kernel_key and parts[2] == sha:
+            return float(parts[1])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the fp64 oracle on the host
+# ---------------------------------------------------------------------------
+
+def oracle_sample(wl_light, rows, expert_cache):
+    import oracle
+    spec = wl_light["spec"]
+    xv = wl_light["x"][rows]
+    shared = [(lambda s=s: expert_cache[("s", s)]) for s in range(spec.n_shared)]
+    return oracle.layer_forward(xv, wl_light["wr"], spec.score, spec.top_k,
+                                lambda e: expert_cache[("r", e)], spec.E, shared,
+                                sel_bias=wl_light["bias"])
+
+
+def light_workload(name, seed=0):
+    """Activations, router and bias of a named workload (no expert weights)."""
+    import torch  # noqa: F401
+    from sparse_expert_moe_b200 import inputs
+    import oracle
+    spec = inputs.SPECS[name]
+    rec = inputs.load_recipe(name)
+    bias = rec.get("sel_bias")
+    if bias is None and name in inputs.BIAS_SOURCE:
+        bias = inputs.load_recipe(inputs.BIAS_SOURCE[name]).get("sel_bias")
+    if bias is None:
+        b = inputs.draw_sel_bias(spec, seed)
+        bias = None if b is None else b.numpy()
+    x32 = inputs._draw_x_fp32(spec, seed, rec.get("redraw"))
+    x, xs = inputs.encode_act(spec, x32)
+    if spec.act == "e4m3":
+        import torch as _t
+        xv = oracle.dequantize_blocks(x.view(_t.uint8).numpy(), xs.numpy(), 1, 128)
+    else:
+        xv = x.double().numpy()
+    wr = inputs.draw_router(spec, seed).double().numpy()
+    return {"spec": spec, "x": xv, "wr": wr,
+            "bias": None if bias is None else np.asarray(bias, np.float64)}
+
+
+def expert_values(spec, seed, keys, host_weights=None):
+    """fp64 values of the experts in `keys` ((kind, index) pairs)."""
+    from sparse_expert_moe_b200 import inputs
+    import oracle
+    import torch
+    out = {}
+    for kind, e in keys:
+        if host_weights is not None:
+            w13 = host_weights["ws13" if kind == "s" else "w13"][e]
+            w2 = host_weights["ws2" if kind == "s" else "w2"][e]
+            s13 = host_weights.get("ws13_s" if kind == "s" else "w13_s")
+            s2 = host_weights.get("ws2_s" if kind == "s" else "w2_s")
+            s13 = None if s13 is None else s13[e]
+            s2 = None if s2 is None else s2[e]
+        else:
+            w13, s13, w2, s2 = inputs.draw_expert(spec, seed, e, kind == "s")
+        if s13 is None:
+            out[(kind, e)] = (w13.double().numpy(), w2.double().numpy())
+        else:
+            out[(kind, e)] = (
+                oracle.dequantize_blocks(w13.view(torch.uint8).numpy(), s13.numpy(), 128, 128),
+                oracle.dequantize_blocks(w2.view(torch.uint8).numpy(), s2.numpy(), 128, 128))
+    return out
+
+
+def needed_experts(light, rows):
+    import oracle
+    spec = light["spec"]
+    L = oracle.router_logits(light["x"][rows], light["wr"])
+    idx, _ = oracle.route(L, spec.score, spec.top_k, light["bias"])
+    keys = sorted({("r", int(e)) for e in np.unique(idx)})
+    return keys + [("s", s) for s in range(spec.n_shared)]
+
+
+def time_oracle(light, rows, cache):
+    t0 = time.perf_counter()
+    oracle_sample(light, rows, cache)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(name, host_weights=None, target_s=15.0):
+    """The oracle as it stands on a bounded sample of the workload's tokens (rank 0 only)."""
+    light = light_workload(name)
+    spec = light["spec"]
+    # grow the sample until one run takes a sizeable share of the budget
+    n = 1
+    keys = needed_experts(light, np.arange(n))
+    cache = expert_values(spec, 0, keys, host_weights)
+    dt = time_oracle(light, np.arange(n), cache)
+    while dt < target_s / 3 and n * 2 <= spec.T:
+        n *= 2
+        keys = needed_experts(light, np.arange(n))
+        cache = expert_values(spec, 0, keys, host_weights)
+        dt = time_oracle(light, np.arange(n), cache)
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {n} tokens of {name} (fp64 NumPy oracle, {len(keys)} experts "
+                      f"upcast per run; {dt:.2f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    light = light_workload(args.workload)
+    spec = light["spec"]
+    rows = np.arange(1)
+    cache = expert_values(spec, 0, needed_experts(light, rows))
+    # each step: the oracle on one token of the workload (the experts' fp64 values prepared
+    # once, outside the timing)
+    for _ in range(args.warmup):
+        time_oracle(light, rows, cache)
+    t = [time_oracle(light, rows, cache) for _ in range(args.steps)]
+    total = sum(t)
+    value = len(rows) * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_tokens_per_step": len(rows)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"1 token of {args.workload} per step, fp64 NumPy oracle"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from sparse_expert_moe_b200 import inputs, moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    name = args.workload
+    wl = inputs.load_workload(name)
+    spec = wl.spec
+    layer = moe.DeviceLayer.from_workload(wl, dev)
+    x = wl.x.to(dev)
+    xs = None if wl.x_scale is None else wl.x_scale.to(dev)
+    y = layer.output(dev)
+    idx = torch.empty((spec.T, spec.top_k), dtype=torch.int32, device=dev)
+    gw = torch.empty((spec.T, spec.top_k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        layer.forward(x, xs, y, idx, gw)
+    torch.cuda.synchronize(dev)
+    if moe.moe_read_device_status(layer.ws) != 0:
+        raise SystemExit("device status set during warm-up")
+
+    # timed steps: stage events recorded in place
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)   # create the events before they are handed to the library
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(K):
+            moe.moe_layer_forward_staged(layer.cfg, layer.weights, x, xs, y, idx, gw, layer.ws, evs[i],
+                                         stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = max_over_ranks(start.elapsed_time(end))
+    ms_step = ms_total / K
+    stage_ms = {s: 0.0 for s in moe.STAGES}
+    for row in evs:
+        for j, s in enumerate(moe.STAGES):
+            stage_ms[s] += row[j].elapsed_time(row[j + 1]) / K
+    status = moe.moe_read_device_status(layer.ws)
+
+    # end to end through the public call: pinned host in, pinned host out, every step
+    x_host = wl.x.pin_memory() if wl.x.dtype != torch.float8_e4m3fn else wl.x.view(torch.uint8).pin_memory()
+    xs_host = None if wl.x_scale is None else wl.x_scale.pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = x if wl.x.dtype != torch.float8_e4m3fn else x.view(torch.uint8)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K):
+        x_dev.copy_(x_host, non_blocking=True)
+        if xs_host is not None:
+            xs.copy_(xs_host, non_blocking=True)
+        layer.forward(x, xs, y, idx, gw)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / K
+    h2d = x_host.numel() * x_host.element_size() + (0 if xs_host is None else xs_host.numel() * 4)
+    d2h = y_host.numel() * y_host.element_size()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    offsets = layer.ws  # group offsets live in the workspace; read them via a fresh routing
+    idx_np = idx.cpu().numpy()
+    sizes = np.bincount(idx_np.ravel(), minlength=spec.E)
+    off = np.concatenate([[0], np.cumsum(sizes)])
+    wm = work_model(spec, off)
+    peaks, peak_src = load_peaks()
+    bound = bound_of(name)
+    if bound == "hbm":
+        dom = "ffn1"
+        achieved = wm["ffn1_bytes"] / (stage_ms["ffn1"] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+        units_note = f"{wm['touched']} touched routed experts + {spec.n_shared} shared: W13 bytes, " \
+                     "token rows read once, h written once"
+    else:
+        dom = "ffn1"
+        achieved = wm["ffn1_flops"] / (stage_ms["ffn1"] * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        if spec.weight == "e4m3":
+            peak *= 2.0   # nominal fp8 : bf16 ratio of the dense tensor-core peaks
+        unit = "TFLOP/s"
+        units_note = "2 * (T*k + S*T) * 2I * d"
+    tokens = spec.T * world
+    value = tokens / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if spec.weight == "e4m3" else "bf16", "data": "synthetic",
+        "config": {"workload": name, "T": spec.T, "d_model": spec.d_model, "E": spec.E,
+                   "top_k": spec.top_k, "d_ff": spec.d_ff, "n_shared": spec.n_shared,
+                   "score": spec.score, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: each step streams "
+                         f"{wm['layer_weight_bytes'] / 1e9:.1f} GB of expert weights"},
+        "roofline": {"bound": bound, "kernel": f"{dom} (grouped_gemm_kernel<1>)",
+                     "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": unit,
+                     "frac": achieved / peak, "traffic": read_traffic(f"ffn1_{name}"),
+                     "units": units_note},
+        "layer": {"weight_bytes_touched": wm["layer_weight_bytes"],
+                  "hbm_frac_layer": wm["layer_weight_bytes"] / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                  "tflops_layer": wm["layer_flops"] / (ms_step * 1e-3) / 1e12,
+                  "touched_experts": wm["touched"]},
+        "stages_ms": stage_ms,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clocks.summary(),
+        "device_status": status,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        host = {n: getattr(wl, n) for n in ("w13", "w2", "ws13", "ws2", "w13_s", "w2_s", "ws13_s",
+                                            "ws2_s")}
+        line["cpu_baseline"] = cpu_baseline(name, host)
+    elif world > 1:
+        line["cpu_baseline"] = None
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

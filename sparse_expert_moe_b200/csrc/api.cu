@@ -1,0 +1,465 @@
+// api.cu -- the C ABI declared in include/moe.h: host-side validation,
+// workspace carving, TMA descriptor encoding and the launch sequence.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeaderBytes = 256;
+// header words
+constexpr int kHdrStatus = 0;
+constexpr int kHdrPermuteDone = 1;
+constexpr int kHdrNChunks = 2;
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+// Byte offsets of every workspace region for one configuration.
+struct Layout {
+  size_t logits, topk_idx, topk_w, offsets, chunk_counts, perm_token, inv_perm, x_perm, chunks, h,
+      y_rows, x_bf16, wr_bf16, w13_bf16, w2_bf16, a_bf16, total;
+  int64_t R, rows_all, n_chunk_max;
+
+  explicit Layout(const moe_config& c) {
+    const int64_t T = c.T, d = c.d_model, E = c.E, k = c.top_k, I = c.d_ff, S = c.n_shared;
+    R = T * k;
+    rows_all = R + S * T;
+    n_chunk_max = max_chunks(rows_all, E + S);
+    const bool f32 = c.act == MOE_F32;
+    size_t o = kHeaderBytes;
+    auto take = [&](size_t bytes) {
+      const size_t at = o;
+      o = align_up(o + bytes);
+      return at;
+    };
+    logits = take(sizeof(float) * T * E);
+    topk_idx = take(sizeof(int32_t) * R);
+    topk_w = take(sizeof(float) * R);
+    offsets = take(sizeof(int32_t) * (E + 1));
+    chunk_counts = take(sizeof(int32_t) * permute_chunks(static_cast<int>(T)) * E);
+    perm_token = take(sizeof(int32_t) * R);
+    inv_perm = take(sizeof(int32_t) * R);
+    x_perm = take(2 * R * d);
+    chunks = take(sizeof(Chunk) * n_chunk_max);
+    h = take(2 * rows_all * I);
+    y_rows = take(2 * rows_all * d);
+    x_bf16 = take(f32 ? 2 * T * d : 0);
+    wr_bf16 = take(f32 ? 2 * E * d : 0);
+    w13_bf16 = take(f32 ? 2 * (E + S) * 2 * I * d : 0);
+    w2_bf16 = take(f32 ? 2 * (E + S) * d * I : 0);
+    a_bf16 = take(f32 ? 2 * rows_all * d : 0);
+    total = o;
+  }
+};
+
+template <class T>
+inline T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+inline int* status_word(void* ws) { return at<int>(ws, kHdrStatus * sizeof(int)); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d_model <= 0 || c->E <= 0 || c->top_k <= 0 || c->d_ff <= 0 ||
+      c->n_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID_BIAS) return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->E || c->top_k > 16 || c->E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (c->d_model % 128 || c->d_ff % 128 || c->d_model > 16384 || c->d_ff > 16384)
+    return MOE_ERR_UNSUPPORTED;
+  if (c->n_shared > 8 || (c->n_shared > 0 && c->d_ff_shared != c->d_ff)) return MOE_ERR_UNSUPPORTED;
+  const int64_t rows_all = static_cast<int64_t>(c->T) * (c->top_k + c->n_shared);
+  if (rows_all >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  const bool fam_bf16 = c->act == MOE_BF16 && c->weight == MOE_BF16;
+  const bool fam_f32 = c->act == MOE_F32 && c->weight == MOE_F32;
+  if (!(fam_bf16 || fam_f32)) return MOE_ERR_UNSUPPORTED;
+  if (c->out != MOE_BF16 && c->out != MOE_F32) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols == 0) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+// The two expert GEMMs over a chunk list already planned into the workspace.
+// seg 0: routed (a0 rows, w13_0 / w2_0 with G0 groups); seg 1: shared (a1 rows,
+// w13_1 / w2_1 with S groups) or absent.  h and y have rows_all rows.
+moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a0, int64_t a0_rows,
+                   const void* w13_0, const void* w2_0, int64_t G0, const void* a1, int64_t a1_rows,
+                   const void* w13_1, const void* w2_1, int64_t S, int64_t rows_all, void* y,
+                   cudaStream_t s, cudaEvent_t* ev = nullptr) {
+  const int64_t d = c.d_model, I = c.d_ff;
+  void* h = at<void>(ws, L.h);
+  GemmLaunch g{};
+  g.chunks = at<Chunk>(ws, L.chunks);
+  g.n_chunks = at<int32_t>(ws, kHdrNChunks * sizeof(int));
+  g.status = status_word(ws);
+  g.num_sms = num_sms();
+
+  g.mode = kFFN1;
+  if (!make_tmap_bf16(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) ||
+      !make_tmap_bf16(&g.tmap[0], a0, a0_rows, d, 16))
+    return MOE_ERR_CUDA;
+  if (S > 0) {
+    if (!make_tmap_bf16(&g.wmap[1], w13_1, S * 2 * I, d, 128) ||
+        !make_tmap_bf16(&g.tmap[1], a1, a1_rows, d, 16))
+      return MOE_ERR_CUDA;
+  } else {
+    g.wmap[1] = g.wmap[0];
+    g.tmap[1] = g.tmap[0];
+  }
+  g.n_mblk = static_cast<int>(I / 128);
+  g.k_blocks = static_cast<int>(d / 64);
+  g.w_rows_per_group = static_cast<int>(2 * I);
+  g.up_offset = static_cast<int>(I);
+  g.m_valid = static_cast<int>(I);
+  g.out = h;
+  g.ld_out = static_cast<int>(I);
+  moe_status st = cuda_status(launch_gemm(g, s));
+  if (st != MOE_OK) return st;
+  if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
+
+  g.mode = kFFN2;
+  if (!make_tmap_bf16(&g.wmap[0], w2_0, G0 * d, I, 128) ||
+      !make_tmap_bf16(&g.tmap[0], h, rows_all, I, 16))
+    return MOE_ERR_CUDA;
+  if (S > 0) {
+    if (!make_tmap_bf16(&g.wmap[1], w2_1, S * d, I, 128)) return MOE_ERR_CUDA;
+  } else {
+    g.wmap[1] = g.wmap[0];
+  }
+  g.tmap[1] = g.tmap[0];
+  g.n_mblk = static_cast<int>(d / 128);
+  g.k_blocks = static_cast<int>(I / 64);
+  g.w_rows_per_group = static_cast<int>(d);
+  g.up_offset = 0;
+  g.m_valid = static_cast<int>(d);
+  g.out = y;
+  g.ld_out = static_cast<int>(d);
+  st = cuda_status(launch_gemm(g, s));
+  if (st != MOE_OK) return st;
+  if (ev) st = cuda_status(cudaEventRecord(ev[1], s));
+  return st;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  const moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  *bytes = Layout(*cfg).total;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const float* logits, const float* sel_bias,
+                     int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  const float* bias = cfg->score == MOE_SCORE_SIGMOID_BIAS ? sel_bias : nullptr;
+  return cuda_status(launch_route(logits, bias, cfg->T, cfg->E, cfg->top_k, cfg->score, topk_idx,
+                                  topk_w, stream));
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                       const float* x_scale, void* x_perm, float* x_perm_scale,
+                       int32_t* perm_token, int32_t* inv_perm, int32_t* group_offsets, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!group_offsets || !ws) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!topk_idx || !x || !x_perm || !perm_token || !inv_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  const Layout L(*cfg);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const int elem = cfg->act == MOE_F32 ? 4 : 2;
+  return cuda_status(launch_permute(topk_idx, cfg->T, cfg->E, cfg->top_k, x, cfg->d_model * elem,
+                                    nullptr, 0, x_perm, nullptr, perm_token, inv_perm,
+                                    group_offsets, at<int32_t>(ws, L.chunk_counts),
+                                    at<unsigned>(ws, kHdrPermuteDone * sizeof(int)),
+                                    status_word(ws), stream));
+}
+
+moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_t* group_offsets,
+                           int32_t n_rows, const void* a, const float* a_scale, const void* w13,
+                           const float* w13_s, const void* w2, const float* w2_s, void* y,
+                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)a_scale;
+  (void)w13_s;
+  (void)w2_s;
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (n_groups <= 0 || n_groups > 1024 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (!group_offsets || !a || !w13 || !w2 || !y || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w13) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  const Layout L(*cfg);
+  if (n_rows > L.rows_all) return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (n_rows == 0) return MOE_OK;
+  const int64_t d = cfg->d_model, I = cfg->d_ff;
+  const void* a_b = a;
+  const void* w13_b = w13;
+  const void* w2_b = w2;
+  if (cfg->act == MOE_F32) {
+    if (n_groups > cfg->E + cfg->n_shared) return MOE_ERR_UNSUPPORTED;
+    st = cuda_status(launch_f32_to_bf16(static_cast<const float*>(a), at<void>(ws, L.a_bf16),
+                                        static_cast<size_t>(n_rows) * d, stream));
+    if (st == MOE_OK)
+      st = cuda_status(launch_f32_to_bf16(static_cast<const float*>(w13), at<void>(ws, L.w13_bf16),
+                                          static_cast<size_t>(n_groups) * 2 * I * d, stream));
+    if (st == MOE_OK)
+      st = cuda_status(launch_f32_to_bf16(static_cast<const float*>(w2), at<void>(ws, L.w2_bf16),
+                                          static_cast<size_t>(n_groups) * d * I, stream));
+    if (st != MOE_OK) return st;
+    a_b = at<void>(ws, L.a_bf16);
+    w13_b = at<void>(ws, L.w13_bf16);
+    w2_b = at<void>(ws, L.w2_bf16);
+  }
+  st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, at<Chunk>(ws, L.chunks),
+                               at<int32_t>(ws, kHdrNChunks * sizeof(int)), status_word(ws), stream));
+  if (st != MOE_OK) return st;
+  return run_ffn(*cfg, L, ws, a_b, n_rows, w13_b, w2_b, n_groups, nullptr, 0, nullptr, nullptr, 0,
+                 n_rows, y, stream);
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* inv_perm,
+                       const float* topk_w, const void* y_shared, void* y, cudaStream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y_perm || !inv_perm || !topk_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(y) || !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
+  const int R = cfg->T * cfg->top_k;
+  return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_shared, y_shared ? 1 : 0, cfg->T,
+                                    cfg->d_model, cfg->top_k, R, cfg->out == MOE_F32, y, stream));
+}
+
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The whole layer.  When `ev` is non-null, ev[0..7] are recorded on the stream
+// before the router GEMM and after each of: router GEMM, route, permute, plan,
+// FFN1, FFN2, combine.
+moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, const void* x,
+                              const float* x_scale, void* y, int32_t* topk_idx_out,
+                              float* topk_w_out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                              cudaEvent_t* ev) {
+  (void)x_scale;
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!wts || !ws) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  if (!x || !y || !wts->wr || !wts->w13 || !wts->w2) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!wts->ws13 || !wts->ws2)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(wts->wr) || !aligned16(wts->w13) ||
+      !aligned16(wts->w2) || !aligned16(wts->ws13) || !aligned16(wts->ws2))
+    return MOE_ERR_INVALID_ARG;
+  const Layout L(c);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const int64_t T = c.T, d = c.d_model, E = c.E, I = c.d_ff, S = c.n_shared;
+  const int64_t R = L.R;
+  cudaStream_t s = stream;
+  int* status = status_word(ws);
+  auto mark = [&](int i) {
+    return ev ? cuda_status(cudaEventRecord(ev[i], s)) : MOE_OK;
+  };
+
+  // f32 family: round every input to bf16 once, into the workspace
+  const void* x_b = x;
+  const void* wr_b = wts->wr;
+  const void* w13_b = wts->w13;
+  const void* w2_b = wts->w2;
+  const void* ws13_b = wts->ws13;
+  const void* ws2_b = wts->ws2;
+  if (c.act == MOE_F32) {
+    auto conv = [&](const void* src, size_t off, size_t n) {
+      return cuda_status(launch_f32_to_bf16(static_cast<const float*>(src), at<void>(ws, off), n, s));
+    };
+    st = conv(x, L.x_bf16, T * d);
+    if (st == MOE_OK) st = conv(wts->wr, L.wr_bf16, E * d);
+    if (st == MOE_OK) st = conv(wts->w13, L.w13_bf16, E * 2 * I * d);
+    if (st == MOE_OK) st = conv(wts->w2, L.w2_bf16, E * d * I);
+    if (st == MOE_OK && S > 0) st = conv(wts->ws13, L.w13_bf16 + 2 * E * 2 * I * d, S * 2 * I * d);
+    if (st == MOE_OK && S > 0) st = conv(wts->ws2, L.w2_bf16 + 2 * E * d * I, S * d * I);
+    if (st != MOE_OK) return st;
+    x_b = at<void>(ws, L.x_bf16);
+    wr_b = at<void>(ws, L.wr_bf16);
+    w13_b = at<void>(ws, L.w13_bf16);
+    w2_b = at<void>(ws, L.w2_bf16);
+    ws13_b = at<char>(ws, L.w13_bf16) + 2 * E * 2 * I * d;
+    ws2_b = at<char>(ws, L.w2_bf16) + 2 * E * d * I;
+  }
+
+  // 1. router GEMM: logits[T, E] = x Wr^T (fp32)
+  float* logits = at<float>(ws, L.logits);
+  if ((st = mark(0)) != MOE_OK) return st;
+  {
+    GemmLaunch g{};
+    g.mode = kRouter;
+    if (!make_tmap_bf16(&g.wmap[0], wr_b, E, d, 128) || !make_tmap_bf16(&g.tmap[0], x_b, T, d, 16))
+      return MOE_ERR_CUDA;
+    g.wmap[1] = g.wmap[0];
+    g.tmap[1] = g.tmap[0];
+    g.router_T = static_cast<int>(T);
+    g.n_mblk = static_cast<int>((E + 127) / 128);
+    g.k_blocks = static_cast<int>(d / 64);
+    g.m_valid = static_cast<int>(E);
+    g.out = logits;
+    g.ld_out = static_cast<int>(E);
+    g.status = status;
+    g.num_sms = num_sms();
+    st = cuda_status(launch_gemm(g, s));
+    if (st != MOE_OK) return st;
+  }
+  if ((st = mark(1)) != MOE_OK) return st;
+
+  // 2. route
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
+  float* gate = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
+  const float* bias = c.score == MOE_SCORE_SIGMOID_BIAS ? wts->sel_bias : nullptr;
+  st = cuda_status(launch_route(logits, bias, c.T, c.E, c.top_k, c.score, idx, gate, s));
+  if (st != MOE_OK) return st;
+  if ((st = mark(2)) != MOE_OK) return st;
+
+  // 3. permute (bf16 rows)
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm_token = at<int32_t>(ws, L.perm_token);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  void* x_perm = at<void>(ws, L.x_perm);
+  st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(d * 2), nullptr, 0,
+                                  x_perm, nullptr, perm_token, inv_perm, offsets,
+                                  at<int32_t>(ws, L.chunk_counts),
+                                  at<unsigned>(ws, kHdrPermuteDone * sizeof(int)), status, s));
+  if (st != MOE_OK) return st;
+  if ((st = mark(3)) != MOE_OK) return st;
+
+  // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs
+  st = cuda_status(launch_plan(offsets, c.E, static_cast<int>(R), c.n_shared, c.T,
+                               static_cast<int>(R), at<Chunk>(ws, L.chunks),
+                               at<int32_t>(ws, kHdrNChunks * sizeof(int)), status, s));
+  if (st != MOE_OK) return st;
+  if ((st = mark(4)) != MOE_OK) return st;
+  void* y_rows = at<void>(ws, L.y_rows);
+  st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows, s,
+               ev ? ev + 5 : nullptr);
+  if (st != MOE_OK) return st;
+
+  // 7. combine
+  const void* y_shared = S > 0 ? static_cast<const void*>(at<char>(ws, L.y_rows) + 2 * R * d) : nullptr;
+  st = cuda_status(launch_combine(y_rows, inv_perm, gate, y_shared, c.n_shared, c.T, c.d_model,
+                                  c.top_k, static_cast<int>(R), c.out == MOE_F32, y, s));
+  if (st != MOE_OK) return st;
+  return mark(7);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* wts, const void* x,
+                             const float* x_scale, void* y, int32_t* topk_idx_out,
+                             float* topk_w_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return layer_forward_impl(cfg, wts, x, x_scale, y, topk_idx_out, topk_w_out, ws, ws_bytes, stream,
+                            nullptr);
+}
+
+moe_status moe_layer_forward_staged(const moe_config* cfg, const moe_weights* wts, const void* x,
+                                    const float* x_scale, void* y, int32_t* topk_idx_out,
+                                    float* topk_w_out, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream, cudaEvent_t* stage_events) {
+  if (!stage_events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 8; ++i)
+    if (!stage_events[i]) return MOE_ERR_INVALID_ARG;
+  return layer_forward_impl(cfg, wts, x, x_scale, y, topk_idx_out, topk_w_out, ws, ws_bytes, stream,
+                            stage_events);
+}
+
+moe_status moe_read_device_status(const void* ws, cudaStream_t stream, moe_status* out) {
+  if (!ws || !out) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  *out = static_cast<moe_status>(v);
+  return MOE_OK;
+}
+
+moe_status moe_reset_device_status(void* ws, cudaStream_t stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, stream));
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_INDEX: return "device: index or offset out of range";
+    case MOE_ERR_TIMEOUT: return "device: bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

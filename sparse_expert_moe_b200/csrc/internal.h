@@ -1,0 +1,83 @@
+// internal.h -- declarations shared by the library's translation units (host side).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+
+namespace moe {
+
+// One group chunk of at most kChunkRows token rows, as produced by the tile
+// planner and consumed by the grouped GEMM kernels.
+//   seg    0 = routed groups (rows of the permuted activations),
+//          1 = shared experts (rows of the unpermuted activations)
+//   group  group (expert) index inside the segment: selects the weights
+//   b_row  first row of the token operand (x_perm / x / h) the chunk reads
+//   o_row  first row of the output (h / y) the chunk writes
+//   nrows  rows in the chunk (1..kChunkRows)
+struct Chunk {
+  int32_t seg, group, b_row, o_row, nrows, pad0, pad1, pad2;
+};
+
+constexpr int kChunkRows = 128;   // tokens per GEMM tile (UMMA N <= 128)
+constexpr int kMaxGroups = 1024 + 8;
+
+// Upper bound on the chunks of `rows` rows spread over `groups` groups.
+inline int64_t max_chunks(int64_t rows, int64_t groups) {
+  return rows / kChunkRows + groups + 1;
+}
+
+// ---------------------------------------------------------------- kernels
+cudaError_t launch_route(const float* logits, const float* sel_bias, int T, int E, int k,
+                         int score, int32_t* topk_idx, float* topk_w, cudaStream_t s);
+
+// Permutation.  `chunk_counts` holds ceil(T / 256) * E ints; `done` one zeroed
+// counter (left zero on exit).
+cudaError_t launch_permute(const int32_t* topk_idx, int T, int E, int k, const void* x,
+                           int row_bytes, const float* x_scale, int scale_cols, void* x_perm,
+                           float* x_perm_scale, int32_t* perm_token, int32_t* inv_perm,
+                           int32_t* offsets, int32_t* chunk_counts, unsigned* done, int* status,
+                           cudaStream_t s);
+inline int permute_chunks(int T) { return (T + 255) / 256; }
+
+// Tile planner: routed groups (device offsets [G+1], rows <= n_rows) followed
+// by n_shared groups of T rows each (token rows 0..T-1 of the unpermuted
+// activations, output rows shared_o_row + s*T).  Heavy groups first.
+cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared, int T,
+                        int shared_o_row, Chunk* chunks, int32_t* n_chunks, int* status,
+                        cudaStream_t s);
+
+enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2 };
+
+struct GemmLaunch {
+  int mode;
+  // weight (A) maps per segment and token (B) maps per segment
+  CUtensorMap wmap[2];
+  CUtensorMap tmap[2];
+  const Chunk* chunks;       // device (FFN modes)
+  const int32_t* n_chunks;   // device (FFN modes)
+  int router_T;              // router mode: tokens
+  int n_mblk;                // 128-row weight blocks per group
+  int k_blocks;              // K / 64
+  int w_rows_per_group;      // weight rows per group (FFN1: 2I, FFN2: d)
+  int up_offset;             // FFN1: I
+  int m_valid;               // router: E
+  void* out;
+  int ld_out;
+  int* status;
+  int num_sms;
+};
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s);
+
+// Tensor map of a row-major [rows, cols] matrix of 2-byte elements, box
+// {64 columns, box_rows rows}, 128-byte swizzle.  Returns false on failure.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+
+cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, const float* topk_w,
+                           const void* y_shared, int n_shared, int T, int d, int k, int R,
+                           bool out_f32, void* y, cudaStream_t s);
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, size_t n, cudaStream_t s);
+
+}  // namespace moe

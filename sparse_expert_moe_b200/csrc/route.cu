@@ -1,0 +1,130 @@
+// route.cu -- router top-k and gate weights, one warp per token.
+//
+// Follows the "topk_softmax" step of the moe_ffn pseudocode ("Decoding
+// Trillion-Parameter MoE LLMs", section "Routing: Top-K Experts Plus a Shared
+// Expert") and the sigmoid + selection-bias variant named "auxiliary-loss-free
+// bias routing" ("Chapter 7: Serving Mega MoE at scale").
+//
+// Each lane holds experts lane, lane+32, ... of the token's logit row (coalesced
+// 128-byte loads).  k rounds of a warp-wide arg-max (shuffle butterfly; key
+// descending, equal keys to the lower expert index) pick the slots in order;
+// lane j keeps slot j and computes its gate with one more butterfly.  HBM-bound:
+// the kernel reads T*E*4 bytes and writes T*k*8.
+#include <cfloat>
+#include <climits>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+__device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
+                                                    const float* __restrict__ sel_bias, int T, int E,
+                                                    int k, int score, int32_t* __restrict__ topk_idx,
+                                                    float* __restrict__ topk_w) {
+  const int token = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (token >= T) return;
+  const float* row = logits + static_cast<size_t>(token) * E;
+
+  float key[VPL], lg[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    float l = 0.f, kk = -FLT_MAX;
+    if (e < E) {
+      l = __ldg(row + e);
+      if (score == 0) {
+        kk = l;
+      } else {
+        kk = sigmoidf_(l) + (sel_bias ? __ldg(sel_bias + e) : 0.f);
+      }
+    }
+    lg[i] = l;
+    key[i] = kk;
+  }
+
+  uint32_t taken = 0;
+  int my_idx = 0;
+  float my_logit = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bk = -FLT_MAX;
+    int be = INT_MAX;
+    float bl = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E && !((taken >> i) & 1u) && better(key[i], e, bk, be)) {
+        bk = key[i];
+        be = e;
+        bl = lg[i];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const float ol = __shfl_xor_sync(0xffffffffu, bl, off);
+      if (better(ok, oe, bk, be)) {
+        bk = ok;
+        be = oe;
+        bl = ol;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == j) {
+      my_idx = be;
+      my_logit = bl;
+    }
+  }
+
+  // gates of the selected experts (lanes 0..k-1), fixed-order butterflies
+  float v;
+  if (score == 0) {
+    float m = lane < k ? my_logit : -FLT_MAX;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    v = lane < k ? expf(my_logit - m) : 0.f;
+  } else {
+    v = lane < k ? sigmoidf_(my_logit) : 0.f;
+  }
+  float sum = v;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(token) * k + lane] = my_idx;
+    topk_w[static_cast<size_t>(token) * k + lane] = v / sum;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const float* logits, const float* sel_bias, int T, int E, int k, int score,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int threads = 256;
+  const int blocks = (T + 7) / 8;
+  if (E <= 32)
+    route_kernel<1><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  else if (E <= 64)
+    route_kernel<2><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  else if (E <= 128)
+    route_kernel<4><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  else if (E <= 256)
+    route_kernel<8><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  else if (E <= 512)
+    route_kernel<16><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  else
+    route_kernel<32><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

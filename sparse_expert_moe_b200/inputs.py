@@ -5,7 +5,8 @@ and ``smoke()``.  It holds none of the layer's arithmetic: it only draws
 random numbers, encodes the drawn values in the storage types the layer
 consumes (bf16 round-to-nearest-even, e4m3 with power-of-two block scales),
 and applies a stored per-workload recipe (rows to redraw so that routing has a
-score margin, and for the Zipf workloads a fitted selection bias).  Recipes are
+score margin -- consecutive keys among each token's k+1 largest differ by at
+least the margin -- and for the Zipf workloads a fitted selection bias).  Recipes are
 JSON files under ``tests/golden/recipes/``, written by
 ``tests/golden/make_recipes.py``, which computes them with the oracle only.
 
@@ -293,18 +294,35 @@ def make_workload(spec: Spec, seed: int = 0, redraw=None, sel_bias=None, threads
                     ws13, ws13_s, ws2, ws2_s, recipe or {})
 
 
-def load_workload(name: str, seed: int = 0, threads=None, T: Optional[int] = None) -> Workload:
+def _same_weights(a: Spec, b: Spec) -> bool:
+    return (a.family, a.weight, a.E, a.d_model, a.d_ff, a.n_shared) == \
+        (b.family, b.weight, b.E, b.d_model, b.d_ff, b.n_shared)
+
+
+def load_workload(name: str, seed: int = 0, threads=None, T: Optional[int] = None,
+                  reuse: Optional[Workload] = None) -> Workload:
     """A named workload with its stored recipe applied (seed 0 recipes are committed).
 
-    ``T`` may shrink the token count (rows 0..T-1 of the same draw).
+    ``T`` may shrink the token count (rows 0..T-1 of the same draw).  ``reuse``: a
+    workload of the same weight family and seed whose expert tensors are taken as they
+    are (expert draws depend only on family, seed, index and storage type).
     """
     spec = SPECS[name]
     recipe = load_recipe(name) if seed == 0 else {}
     bias = recipe.get("sel_bias")
     if bias is None and name in BIAS_SOURCE and seed == 0:
         bias = load_recipe(BIAS_SOURCE[name]).get("sel_bias")
-    w = make_workload(spec, seed, redraw=recipe.get("redraw"), sel_bias=bias, threads=threads,
-                      recipe=recipe)
+    if reuse is not None and reuse.seed == seed and _same_weights(reuse.spec, spec):
+        x, x_scale = encode_act(spec, _draw_x_fp32(spec, seed, recipe.get("redraw")))
+        if bias is None:
+            sb = draw_sel_bias(spec, seed)
+        else:
+            sb = torch.tensor(np.asarray(bias, np.float32))
+        w = Workload(spec, seed, x, x_scale, draw_router(spec, seed), sb, reuse.w13, reuse.w13_s,
+                     reuse.w2, reuse.w2_s, reuse.ws13, reuse.ws13_s, reuse.ws2, reuse.ws2_s, recipe)
+    else:
+        w = make_workload(spec, seed, redraw=recipe.get("redraw"), sel_bias=bias, threads=threads,
+                          recipe=recipe)
     if T is not None and T != spec.T:
         w.spec = replace(spec, T=T)
         w.x = w.x[:T].contiguous()

@@ -3,9 +3,9 @@
 A recipe holds what the input generator cannot derive without the layer's
 arithmetic:
 
-* ``redraw``: activation rows that were redrawn (row, attempt) until the
-  fp64 selection keys of every token have a gap of at least ``margin``
-  between the k-th and the (k+1)-th largest key, so that the selection is
+* ``redraw``: activation rows that were redrawn (row, attempt) until, for
+  every token, consecutive fp64 selection keys among its k+1 largest differ
+  by at least ``margin``, so that the selection and the slot order are both
   well defined under fp32 accumulation;
 * ``sel_bias`` (Zipf workloads): the per-expert selection bias fitted so that
   the realised expert loads follow the target loads of Zipf(1.1) sampling
@@ -48,11 +48,13 @@ def _keys(spec, xv, wr, bias):
 
 
 def _gaps(spec, keys):
+    """Smallest gap between consecutive keys among each token's k+1 largest: the selection
+    and the slot order are then both decided by more than ``margin``."""
     s = -np.sort(-keys, axis=1)
-    k = spec.top_k
-    if k >= spec.E:
+    m = min(spec.top_k + 1, spec.E)
+    if m < 2:
         return np.full(keys.shape[0], np.inf)
-    return s[:, k - 1] - s[:, k]
+    return (s[:, : m - 1] - s[:, 1:m]).min(axis=1)
 
 
 def fit_bias(spec, xv, wr, target):

@@ -1,0 +1,175 @@
+"""moe_grouped_ffn, moe_combine and moe_layer_forward on the GPU against the oracle.
+
+Metric: max relative error ||y - ref||_inf / ||ref||_inf, bar 2e-2 for bf16 (the
+layer's stated tolerance); the oracle is fp64 on the exact input values."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_expert_moe_b200 import inputs, moe
+
+from helpers import margin_workload, max_rel_err, oracle_layer
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL_BF16 = 2e-2
+
+
+def _bf16(a):
+    return inputs.to_bf16(np.asarray(a, np.float32))
+
+
+# ---------------------------------------------------------------------------
+# grouped FFN alone
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("sizes,d,I", [
+    ([5, 0, 1, 130, 16, 17, 0, 128], 256, 256),     # ragged: empty, 1 row, > one 128-row chunk
+    ([300], 128, 384),                               # one group, three chunks, ragged tail
+    ([1, 1, 1, 1], 512, 128),
+])
+def test_grouped_ffn_vs_oracle(sizes, d, I):
+    rng = np.random.default_rng(sum(sizes) + d + I)
+    G = len(sizes)
+    n_rows = sum(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    a = _bf16(rng.standard_normal((n_rows, d)))
+    w13 = _bf16(rng.standard_normal((G, 2 * I, d)) * 0.05)
+    w2 = _bf16(rng.standard_normal((G, d, I)) * 0.05)
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0)
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows, a.to(DEV), None,
+                        w13.to(DEV), None, w2.to(DEV), None, y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    ref = np.zeros((n_rows, d))
+    for g in range(G):
+        lo, hi = offsets[g], offsets[g + 1]
+        if hi > lo:
+            ref[lo:hi] = oracle.swiglu_expert(a[lo:hi].double().numpy(), w13[g].double().numpy(),
+                                              w2[g].double().numpy())
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert max_rel_err(got, ref) < TOL_BF16
+
+
+def test_grouped_ffn_bad_offsets_set_device_status():
+    d, I, G = 128, 128, 3
+    cfg = moe.make_config(8, d, G, 1, I, 0)
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    offsets = torch.tensor([0, 5, 3, 8], dtype=torch.int32, device=DEV)     # decreasing
+    a = torch.zeros((8, d), dtype=torch.bfloat16, device=DEV)
+    w13 = torch.zeros((G, 2 * I, d), dtype=torch.bfloat16, device=DEV)
+    w2 = torch.zeros((G, d, I), dtype=torch.bfloat16, device=DEV)
+    y = torch.zeros((8, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, offsets, 8, a, None, w13, None, w2, None, y, ws)
+    assert moe.moe_read_device_status(ws) == 5
+
+
+# ---------------------------------------------------------------------------
+# combine alone
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,k,d,shared", [(1, 2, 128, False), (77, 8, 7168, True), (64, 16, 256, True)])
+def test_combine_vs_oracle(T, k, d, shared):
+    rng = np.random.default_rng(T * k)
+    R = T * k
+    y_perm = _bf16(rng.standard_normal((R, d)))
+    inv = rng.permutation(R).reshape(T, k).astype(np.int32)
+    w = rng.uniform(0, 1, (T, k)).astype(np.float32)
+    ys = _bf16(rng.standard_normal((T, d))) if shared else None
+    cfg = moe.make_config(T, d, 16, k, 128, 1 if shared else 0)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(cfg, y_perm.to(DEV), torch.from_numpy(inv).to(DEV), torch.from_numpy(w).to(DEV),
+                    None if ys is None else ys.to(DEV), y)
+    ref = oracle.combine(y_perm.double().numpy(), inv, w.astype(np.float64),
+                         None if ys is None else [ys.double().numpy()])
+    got = y.float().cpu().numpy()
+    # one bf16 rounding of an fp32 sum
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5 * np.abs(ref).max())
+
+
+# ---------------------------------------------------------------------------
+# the whole layer
+# ---------------------------------------------------------------------------
+
+def _run_layer(wl, T=None):
+    layer = moe.DeviceLayer.from_workload(wl, DEV, T=T)
+    x = wl.x.to(DEV)
+    xs = None if wl.x_scale is None else wl.x_scale.to(DEV)
+    idx = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.int32, device=DEV)
+    gw = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.float32, device=DEV)
+    y = layer.forward(x, xs, topk_idx=idx, topk_w=gw)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(layer.ws) == 0
+    return layer, y.float().cpu().numpy(), idx.cpu().numpy(), gw.cpu().numpy()
+
+
+def _check_layer(wl, rows=None):
+    layer, y, idx, gw = _run_layer(wl)
+    ref, r = oracle_layer(wl, rows=rows, return_routing=True)
+    if rows is not None:
+        y, idx, gw = y[rows], idx[rows], gw[rows]
+    assert np.array_equal(idx, r["idx"])
+    np.testing.assert_allclose(gw, r["gates"], rtol=1e-5, atol=1e-6)
+    err = max_rel_err(y, ref)
+    assert err < TOL_BF16, err
+    return layer, err
+
+
+def test_layer_tiny_config():
+    wl = inputs.load_workload("tiny")
+    _check_layer(wl)
+
+
+@pytest.mark.parametrize("T,d,E,k,I,S,score", [
+    (1, 128, 8, 2, 128, 1, "sigmoid_bias"),
+    (63, 256, 16, 4, 256, 1, "softmax"),
+    (200, 384, 32, 8, 256, 2, "sigmoid_bias"),
+    (130, 128, 1, 1, 128, 0, "softmax"),          # E = 1, k = 1: a dense SwiGLU FFN
+    (520, 256, 4, 2, 128, 1, "sigmoid_bias"),     # heavy groups: several 128-row chunks each
+])
+def test_layer_custom(T, d, E, k, I, S, score):
+    spec = inputs.custom_spec(T, d, E, k, I, S, score=score)
+    _check_layer(margin_workload(spec, seed=T))
+
+
+def test_layer_is_deterministic():
+    spec = inputs.custom_spec(300, 256, 16, 4, 256, 1)
+    wl = margin_workload(spec, seed=4)
+    layer = moe.DeviceLayer.from_workload(wl, DEV)
+    x = wl.x.to(DEV)
+    a = layer.forward(x).clone()
+    b = layer.forward(x).clone()
+    assert torch.equal(a, b)
+
+
+_FULL = {}
+
+
+def _full_workload(name):
+    """Full-size workloads share their expert draws within a weight family."""
+    prev = _FULL.get(inputs.SPECS[name].family)
+    wl = inputs.load_workload(name, reuse=prev)
+    _FULL.clear()
+    _FULL[wl.spec.family] = wl
+    return wl
+
+
+@pytest.mark.slow
+def test_layer_r1_decode_full():
+    """The DeepSeek-R1-shaped decode layer, every token checked."""
+    wl = _full_workload("r1_decode")
+    _check_layer(wl)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["r1_prefill", "kimi"])
+def test_layer_full_size_sampled(name):
+    """Full-size prefill-shaped layers in the launch configuration the bench times; the
+    oracle evaluates a sample of tokens one by one (the layer is per-token)."""
+    wl = _full_workload(name)
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(wl.spec.T, 12, replace=False))
+    _check_layer(wl, rows=rows)

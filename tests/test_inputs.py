@@ -72,7 +72,8 @@ def test_recipe_margin_and_loads(name):
     w = inputs.Workload(spec, 0, x, xs, wr, b, *([None] * 8))
     keys, idx = _routing_of(w)
     srt = -np.sort(-keys, axis=1)
-    assert np.all(srt[:, spec.top_k - 1] - srt[:, spec.top_k] >= spec.margin)
+    m = min(spec.top_k + 1, spec.E)
+    assert np.all((srt[:, : m - 1] - srt[:, 1:m]).min(axis=1) >= spec.margin)
     assert np.bincount(idx.ravel(), minlength=spec.E).tolist() == rec["realised_loads"]
 
 
@@ -89,3 +90,13 @@ def test_zipf_recipe_summary():
     assert np.corrcoef(np.log(loads + 1), np.log(target + 1))[0, 1] > 0.99
     fp8 = inputs.load_recipe("r1_prefill_fp8")
     assert fp8["margin"] == spec.margin and "sel_bias" not in fp8
+
+
+def test_reuse_gives_identical_expert_tensors():
+    spec = inputs.custom_spec(T=4, d_model=128, E=2, top_k=1, d_ff=128, n_shared=1)
+    a = inputs.make_workload(spec, seed=5, threads=1)
+    for e in range(2):
+        q13, _, q2, _ = inputs.draw_expert(spec, 5, e)
+        assert torch.equal(q13, a.w13[e]) and torch.equal(q2, a.w2[e])
+    q13, _, q2, _ = inputs.draw_expert(spec, 5, 0, shared=True)
+    assert torch.equal(q13, a.ws13[0]) and torch.equal(q2, a.ws2[0])
