@@ -178,19 +178,8 @@ def read_traffic(kernel_key):
 # the reference arm: the fp64 oracle on the host
 # ---------------------------------------------------------------------------
 
-def oracle_sample(wl_light, rows, expert_cache):
-    import oracle
-    spec = wl_light["spec"]
-    xv = wl_light["x"][rows]
-    shared = [(lambda s=s: expert_cache[("s", s)]) for s in range(spec.n_shared)]
-    return oracle.layer_forward(xv, wl_light["wr"], spec.score, spec.top_k,
-                                lambda e: expert_cache[("r", e)], spec.E, shared,
-                                sel_bias=wl_light["bias"])
-
-
 def light_workload(name, seed=0):
     """Activations, router and bias of a named workload (no expert weights)."""
-    import torch  # noqa: F401
     from sparse_expert_moe_b200 import inputs
     import oracle
     spec = inputs.SPECS[name]
@@ -203,73 +192,93 @@ def light_workload(name, seed=0):
         bias = None if b is None else b.numpy()
     x32 = inputs._draw_x_fp32(spec, seed, rec.get("redraw"))
     x, xs = inputs.encode_act(spec, x32)
-    if spec.act == "e4m3":
-        import torch as _t
-        xv = oracle.dequantize_blocks(x.view(_t.uint8).numpy(), xs.numpy(), 1, 128)
-    else:
-        xv = x.double().numpy()
-    wr = inputs.draw_router(spec, seed).double().numpy()
-    return {"spec": spec, "x": xv, "wr": wr,
+    return {"spec": spec, "x": x, "x_scale": xs, "wr": inputs.draw_router(spec, seed),
             "bias": None if bias is None else np.asarray(bias, np.float64)}
 
 
-def expert_values(spec, seed, keys, host_weights=None):
-    """fp64 values of the experts in `keys` ((kind, index) pairs)."""
-    from sparse_expert_moe_b200 import inputs
+def _act_values(light, rows):
     import oracle
     import torch
-    out = {}
-    for kind, e in keys:
-        if host_weights is not None:
-            w13 = host_weights["ws13" if kind == "s" else "w13"][e]
-            w2 = host_weights["ws2" if kind == "s" else "w2"][e]
-            s13 = host_weights.get("ws13_s" if kind == "s" else "w13_s")
-            s2 = host_weights.get("ws2_s" if kind == "s" else "w2_s")
-            s13 = None if s13 is None else s13[e]
-            s2 = None if s2 is None else s2[e]
-        else:
-            w13, s13, w2, s2 = inputs.draw_expert(spec, seed, e, kind == "s")
-        if s13 is None:
-            out[(kind, e)] = (w13.double().numpy(), w2.double().numpy())
-        else:
-            out[(kind, e)] = (
-                oracle.dequantize_blocks(w13.view(torch.uint8).numpy(), s13.numpy(), 128, 128),
-                oracle.dequantize_blocks(w2.view(torch.uint8).numpy(), s2.numpy(), 128, 128))
-    return out
+    x = light["x"][rows]
+    if light["x_scale"] is not None:
+        return oracle.dequantize_blocks(x.view(torch.uint8).numpy(),
+                                        light["x_scale"][rows].numpy(), 1, 128)
+    return x.double().numpy()
+
+
+def _weight_values(w, s):
+    import oracle
+    import torch
+    if s is None:
+        return w.double().numpy()
+    return oracle.dequantize_blocks(w.view(torch.uint8).numpy(), s.numpy(), 128, 128)
 
 
 def needed_experts(light, rows):
     import oracle
     spec = light["spec"]
-    L = oracle.router_logits(light["x"][rows], light["wr"])
+    L = oracle.router_logits(_act_values(light, rows), light["wr"].double().numpy())
     idx, _ = oracle.route(L, spec.score, spec.top_k, light["bias"])
-    keys = sorted({("r", int(e)) for e in np.unique(idx)})
-    return keys + [("s", s) for s in range(spec.n_shared)]
+    return sorted({int(e) for e in np.unique(idx)})
 
 
-def time_oracle(light, rows, cache):
+def stored_experts(spec, seed, routed, host_weights=None):
+    """Storage-typed (bf16 / e4m3 + scales) tensors of the listed routed experts and the
+    shared experts: taken from resident host copies or drawn."""
+    from sparse_expert_moe_b200 import inputs
+    out = {}
+    for kind, ids in (("r", routed), ("s", range(spec.n_shared))):
+        for e in ids:
+            if host_weights is not None:
+                pre = "ws" if kind == "s" else "w"
+                get = lambda n: None if host_weights.get(n) is None else host_weights[n][e]
+                out[(kind, e)] = (get(pre + "13"), get(pre + "13_s"), get(pre + "2"), get(pre + "2_s"))
+            else:
+                out[(kind, e)] = inputs.draw_expert(spec, seed, e, kind == "s")
+    return out
+
+
+def time_oracle(light, rows, stored):
+    """One oracle run on `rows`, timed as it stands: routing, decoding the inputs to fp64
+    (activations and every expert it touches) and the fp64 arithmetic."""
+    import oracle
+    spec = light["spec"]
+
+    def expert(kind, e):
+        w13, s13, w2, s2 = stored[(kind, e)]
+        return _weight_values(w13, s13), _weight_values(w2, s2)
+
     t0 = time.perf_counter()
-    oracle_sample(light, rows, cache)
+    xv = _act_values(light, rows)
+    oracle.layer_forward(xv, light["wr"].double().numpy(), spec.score, spec.top_k,
+                         lambda e: expert("r", e), spec.E,
+                         [(lambda s=s: expert("s", s)) for s in range(spec.n_shared)],
+                         sel_bias=light["bias"])
     return time.perf_counter() - t0
 
 
-def cpu_baseline(name, host_weights=None, target_s=15.0):
-    """The oracle as it stands on a bounded sample of the workload's tokens (rank 0 only)."""
+def cpu_baseline(name, host_weights=None, budget_s=25.0):
+    """The oracle as it stands on a bounded sample of the workload's tokens (rank 0 only):
+    the first n tokens, n the largest power of two (<= T) whose run stays in the budget."""
     light = light_workload(name)
     spec = light["spec"]
-    # grow the sample until one run takes a sizeable share of the budget
     n = 1
-    keys = needed_experts(light, np.arange(n))
-    cache = expert_values(spec, 0, keys, host_weights)
-    dt = time_oracle(light, np.arange(n), cache)
-    while dt < target_s / 3 and n * 2 <= spec.T:
-        n *= 2
-        keys = needed_experts(light, np.arange(n))
-        cache = expert_values(spec, 0, keys, host_weights)
-        dt = time_oracle(light, np.arange(n), cache)
+    rows = np.arange(n)
+    stored = stored_experts(spec, 0, needed_experts(light, rows), host_weights)
+    dt = time_oracle(light, rows, stored)
+    while n * 2 <= spec.T:
+        n2 = n * 2
+        rows2 = np.arange(n2)
+        routed = needed_experts(light, rows2)
+        # cost grows with the experts touched (their fp64 decoding dominates)
+        if dt * (len(routed) + spec.n_shared) / max(len(stored), 1) * 1.2 > budget_s:
+            break
+        stored = stored_experts(spec, 0, routed, host_weights)
+        n, rows = n2, rows2
+        dt = time_oracle(light, rows, stored)
     return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {n} tokens of {name} (fp64 NumPy oracle, {len(keys)} experts "
-                      f"upcast per run; {dt:.2f} s)"}
+            "sample": f"first {n} tokens of {name}: fp64 NumPy oracle incl. decoding "
+                      f"{len(stored)} experts to fp64; {dt:.2f} s"}
 
 
 def run_reference(args):
@@ -279,12 +288,11 @@ def run_reference(args):
     light = light_workload(args.workload)
     spec = light["spec"]
     rows = np.arange(1)
-    cache = expert_values(spec, 0, needed_experts(light, rows))
-    # each step: the oracle on one token of the workload (the experts' fp64 values prepared
-    # once, outside the timing)
+    # inputs drawn outside the timing; each step = the oracle on one token of the workload
+    stored = stored_experts(spec, 0, needed_experts(light, rows))
     for _ in range(args.warmup):
-        time_oracle(light, rows, cache)
-    t = [time_oracle(light, rows, cache) for _ in range(args.steps)]
+        time_oracle(light, rows, stored)
+    t = [time_oracle(light, rows, stored) for _ in range(args.steps)]
     total = sum(t)
     value = len(rows) * args.steps / total
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -294,7 +302,8 @@ def run_reference(args):
             "config": {"workload": args.workload, "sample_tokens_per_step": len(rows)},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                              "kind": "oracle",
-                             "sample": f"1 token of {args.workload} per step, fp64 NumPy oracle"},
+                             "sample": f"token 0 of {args.workload} per step: fp64 NumPy oracle "
+                                       f"incl. decoding its {len(stored)} experts to fp64"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -404,7 +413,6 @@ def run_ours(args):
             dist.destroy_process_group()
         return
 
-    offsets = layer.ws  # group offsets live in the workspace; read them via a fresh routing
     idx_np = idx.cpu().numpy()
     sizes = np.bincount(idx_np.ravel(), minlength=spec.E)
     off = np.concatenate([[0], np.cumsum(sizes)])

@@ -112,7 +112,13 @@ def _check_layer(wl, rows=None):
     if rows is not None:
         y, idx, gw = y[rows], idx[rows], gw[rows]
     assert np.array_equal(idx, r["idx"])
-    np.testing.assert_allclose(gw, r["gates"], rtol=1e-5, atol=1e-6)
+    if wl.spec.act == "f32":
+        # f32 inputs are rounded to bf16 on entry: each product x_i * w_i moves by up to
+        # 2^-8 relative, so a logit by up to sum |x_i w_i| 2^-8 (~6e-3 at d = 128) and a
+        # gate by up to a quarter of the difference of two such errors
+        np.testing.assert_allclose(gw, r["gates"], rtol=0, atol=3e-3)
+    else:
+        np.testing.assert_allclose(gw, r["gates"], rtol=1e-5, atol=1e-6)
     err = max_rel_err(y, ref)
     assert err < TOL_BF16, err
     return layer, err
