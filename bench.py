@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling case: the workload with only this many routed experts "
+                         "(drawn without the stored recipe; not a bench line)")
     return ap.parse_args()
 
 
@@ -342,7 +345,12 @@ def run_ours(args):
         return float(t.item())
 
     name = args.workload
-    wl = inputs.load_workload(name)
+    if args.experts:
+        from dataclasses import replace
+        spec = replace(inputs.SPECS[name], E=args.experts)
+        wl = inputs.make_workload(spec, 0)
+    else:
+        wl = inputs.load_workload(name)
     spec = wl.spec
     layer = moe.DeviceLayer.from_workload(wl, dev)
     x = wl.x.to(dev)
@@ -441,7 +449,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if spec.weight == "e4m3" else "bf16", "data": "synthetic",
-        "config": {"workload": name, "T": spec.T, "d_model": spec.d_model, "E": spec.E,
+        "config": {"workload": name if not args.experts else f"{name} with E={spec.E} (profiling case)",
+                   "T": spec.T, "d_model": spec.d_model, "E": spec.E,
                    "top_k": spec.top_k, "d_ff": spec.d_ff, "n_shared": spec.n_shared,
                    "score": spec.score, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: each step streams "
