@@ -137,6 +137,30 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, c
                        int32_t *perm_token, int32_t *inv_perm, int32_t *group_offsets,
                        void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory to give the library -- for instance a plugin whose host application
+ * owns every device allocation through its own pool, or code on a latency path
+ * where cudaMalloc (which may synchronise the device) is not allowed.  The pages
+ * have no counterpart: it is the same permutation with the same arguments and
+ * results as moe_permute, minus ws / ws_bytes.
+ * Its scratch is a fixed array inside the library (about 1 MiB per GPU that
+ * loads the library, held until the process exits), so it accepts only
+ * ceil(T / 256) * E <= 262144 (for example T <= 65536 with E <= 1024); larger
+ * shapes return MOE_ERR_UNSUPPORTED.  It calls no allocator.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current); make that first call before any stream capture.
+ *  - Every call shares the one array, which keeps the previous call's contents;
+ *    the call clears what must start at zero itself.  Calls whose kernels
+ *    overlap on the GPU (several streams, or several host threads) race on it:
+ *    serialise them.
+ *  - No device status is recorded: pairs with an expert index outside [0, E)
+ *    are dropped (inv_perm = -1, not counted in group_offsets). */
+MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *topk_idx,
+                                       const void *x, const float *x_scale, void *x_perm,
+                                       float *x_perm_scale, int32_t *perm_token,
+                                       int32_t *inv_perm, int32_t *group_offsets,
+                                       cudaStream_t stream);
+
 /* Grouped SwiGLU expert FFN over ragged groups (one expert per group):
  *   y[r] = (silu(a[r] W1_g^T) * (a[r] W3_g^T)) W2_g^T  for rows r of group g.
  *   n_groups        G (<= 1024); group g uses weights w13[g], w2[g]

@@ -115,6 +115,8 @@ int num_sms() {
 
 }  // namespace
 
+moe_status validate_config(const moe_config* c) { return check_config(c); }
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();

@@ -5,7 +5,12 @@
 #include <cuda.h>
 #include <cuda_runtime_api.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
+
+// Host-side configuration checks shared by every entry point (MOE_OK or the error code).
+moe_status validate_config(const moe_config* c);
 
 // One group chunk of at most kChunkRows token rows, as produced by the tile
 // planner and consumed by the grouped GEMM kernels.

@@ -63,6 +63,7 @@ def load_library() -> ctypes.CDLL:
         "moe_workspace_size": [cfgp, ctypes.POINTER(SZ)],
         "moe_route": [cfgp, P, P, P, P, P],
         "moe_permute": [cfgp, P, P, P, P, P, P, P, P, P, SZ, P],
+        "moe_permute_noalloc": [cfgp, P, P, P, P, P, P, P, P, P],
         "moe_grouped_ffn": [cfgp, I32, P, I32, P, P, P, P, P, P, P, P, SZ, P],
         "moe_combine": [cfgp, P, P, P, P, P, P],
         "moe_layer_forward": [cfgp, ctypes.POINTER(MoeWeights), P, P, P, P, P, P, SZ, P],
@@ -145,6 +146,14 @@ def moe_permute(cfg, topk_idx, x, x_scale, x_perm, x_perm_scale, perm_token, inv
         ctypes.byref(cfg), _p(topk_idx), _p(x), _p(x_scale), _p(x_perm), _p(x_perm_scale),
         _p(perm_token), _p(inv_perm), _p(group_offsets), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def moe_permute_noalloc(cfg, topk_idx, x, x_scale, x_perm, x_perm_scale, perm_token, inv_perm,
+                        group_offsets, stream=None):
+    """moe_permute without a workspace (scratch inside the library; see include/moe.h)."""
+    _check("moe_permute_noalloc", load_library().moe_permute_noalloc(
+        ctypes.byref(cfg), _p(topk_idx), _p(x), _p(x_scale), _p(x_perm), _p(x_perm_scale),
+        _p(perm_token), _p(inv_perm), _p(group_offsets), _stream(stream)))
 
 
 def moe_grouped_ffn(cfg, n_groups, group_offsets, n_rows, a, a_scale, w13, w13_s, w2, w2_s, y, ws,
