@@ -24,7 +24,8 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 // Byte offsets of every workspace region for one configuration.
 struct Layout {
   size_t logits, topk_idx, topk_w, offsets, chunk_counts, perm_token, inv_perm, x_perm, chunks, h,
-      y_rows, x_bf16, wr_bf16, w13_bf16, w2_bf16, a_bf16, total;
+      y_rows, x_bf16, wr_bf16, w13_bf16, w2_bf16, a_bf16, x_sf, x_perm_sf, h_sf, a_sf, wsf13, wsf2,
+      total;
   int64_t R, rows_all, n_chunk_max;
 
   explicit Layout(const moe_config& c) {
@@ -33,13 +34,14 @@ struct Layout {
     rows_all = R + S * T;
     n_chunk_max = max_chunks(rows_all, E + S);
     const bool f32 = c.act == MOE_F32;
+    const bool fp8 = c.act == MOE_E4M3;
     size_t o = kHeaderBytes;
     auto take = [&](size_t bytes) {
       const size_t at = o;
       o = align_up(o + bytes);
       return at;
     };
-    logits = take(sizeof(float) * T * E);
+    logits = take(sizeof(float) * router_splits(T, E, d) * T * E);
     topk_idx = take(sizeof(int32_t) * R);
     topk_w = take(sizeof(float) * R);
     offsets = take(sizeof(int32_t) * (E + 1));
@@ -50,11 +52,18 @@ struct Layout {
     chunks = take(sizeof(Chunk) * n_chunk_max);
     h = take(2 * rows_all * I);
     y_rows = take(2 * rows_all * d);
-    x_bf16 = take(f32 ? 2 * T * d : 0);
+    x_bf16 = take(f32 || fp8 ? 2 * T * d : 0);
     wr_bf16 = take(f32 ? 2 * E * d : 0);
     w13_bf16 = take(f32 ? 2 * (E + S) * 2 * I * d : 0);
     w2_bf16 = take(f32 ? 2 * (E + S) * d * I : 0);
     a_bf16 = take(f32 ? 2 * rows_all * d : 0);
+    // FP8: UE8M0 scale factors in the layouts the grouped GEMM's scale warp reads
+    x_sf = take(fp8 ? 4 * (d / 128) * T : 0);
+    x_perm_sf = take(fp8 ? 4 * (d / 128) * R : 0);
+    h_sf = take(fp8 ? 4 * (I / 128) * rows_all : 0);
+    a_sf = take(fp8 ? 4 * (d / 128) * rows_all : 0);
+    wsf13 = take(fp8 ? 16 * (E + S) * (2 * I / 128) * (d / 128) : 0);
+    wsf2 = take(fp8 ? 16 * (E + S) * (d / 128) * (I / 128) : 0);
     total = o;
   }
 };
@@ -81,7 +90,8 @@ moe_status check_config(const moe_config* c) {
   if (rows_all >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   const bool fam_bf16 = c->act == MOE_BF16 && c->weight == MOE_BF16;
   const bool fam_f32 = c->act == MOE_F32 && c->weight == MOE_F32;
-  if (!(fam_bf16 || fam_f32)) return MOE_ERR_UNSUPPORTED;
+  const bool fam_fp8 = c->act == MOE_E4M3 && c->weight == MOE_E4M3;
+  if (!(fam_bf16 || fam_f32 || fam_fp8)) return MOE_ERR_UNSUPPORTED;
   if (c->out != MOE_BF16 && c->out != MOE_F32) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -130,7 +140,108 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols == 0) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
+
+// The FP8 block-scaled expert GEMMs over a chunk list already planned into the
+// workspace.  seg 0: routed rows a0 (token scales a0_sf [d/128][a0_rows]) with
+// weights w13_0 / w2_0 and their UE8M0 block scales wsf13_0 / wsf2_0 (G0 groups);
+// seg 1: shared experts on rows a1 (scales a1_sf) or absent (S = 0).  h (e4m3) and
+// its scales live in the workspace; y has rows_all rows.
+moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const void* a0,
+                       const uint32_t* a0_sf, int64_t a0_rows, const void* w13_0, const void* w2_0,
+                       const uint4* wsf13_0, const uint4* wsf2_0, int64_t G0, const void* a1,
+                       const uint32_t* a1_sf, int64_t a1_rows, const void* w13_1, const void* w2_1,
+                       const uint4* wsf13_1, const uint4* wsf2_1, int64_t S, int64_t rows_all,
+                       void* y, cudaStream_t s, cudaEvent_t* ev = nullptr) {
+  const int64_t d = c.d_model, I = c.d_ff;
+  void* h = at<void>(ws, L.h);
+  uint32_t* h_sf = at<uint32_t>(ws, L.h_sf);
+  GemmLaunch g{};
+  g.chunks = at<Chunk>(ws, L.chunks);
+  g.n_chunks = at<int32_t>(ws, kHdrNChunks * sizeof(int));
+  g.status = status_word(ws);
+  g.num_sms = num_sms();
+
+  g.mode = kFFN1F8;
+  if (!make_tmap_u8(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) || !make_tmap_u8(&g.tmap[0], a0, a0_rows, d, 16))
+    return MOE_ERR_CUDA;
+  g.wsf[0] = wsf13_0;
+  g.tsf[0] = a0_sf;
+  g.tsf_ld[0] = static_cast<int>(a0_rows);
+  g.tsf_rows[0] = static_cast<int>(a0_rows);
+  if (S > 0) {
+    if (!make_tmap_u8(&g.wmap[1], w13_1, S * 2 * I, d, 128) || !make_tmap_u8(&g.tmap[1], a1, a1_rows, d, 16))
+      return MOE_ERR_CUDA;
+    g.wsf[1] = wsf13_1;
+    g.tsf[1] = a1_sf;
+    g.tsf_ld[1] = static_cast<int>(a1_rows);
+    g.tsf_rows[1] = static_cast<int>(a1_rows);
+  } else {
+    g.wmap[1] = g.wmap[0];
+    g.tmap[1] = g.tmap[0];
+    g.wsf[1] = g.wsf[0];
+    g.tsf[1] = g.tsf[0];
+    g.tsf_ld[1] = g.tsf_ld[0];
+    g.tsf_rows[1] = g.tsf_rows[0];
+  }
+  g.n_mblk = static_cast<int>(I / 128);
+  g.k_blocks = static_cast<int>(d / 128);
+  g.w_rows_per_group = static_cast<int>(2 * I);
+  g.wsf_rb_per_group = static_cast<int>(2 * I / 128);
+  g.up_offset = static_cast<int>(I);
+  g.m_valid = static_cast<int>(I);
+  g.out = h;
+  g.ld_out = static_cast<int>(I);
+  g.out_sf = h_sf;
+  g.ld_out_sf = static_cast<int>(rows_all);
+  moe_status st = cuda_status(launch_gemm(g, s));
+  if (st != MOE_OK) return st;
+  if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
+
+  g.mode = kFFN2F8;
+  if (!make_tmap_u8(&g.wmap[0], w2_0, G0 * d, I, 128) || !make_tmap_u8(&g.tmap[0], h, rows_all, I, 16))
+    return MOE_ERR_CUDA;
+  g.wsf[0] = wsf2_0;
+  if (S > 0) {
+    if (!make_tmap_u8(&g.wmap[1], w2_1, S * d, I, 128)) return MOE_ERR_CUDA;
+    g.wsf[1] = wsf2_1;
+  } else {
+    g.wmap[1] = g.wmap[0];
+    g.wsf[1] = g.wsf[0];
+  }
+  g.tmap[1] = g.tmap[0];
+  for (int i = 0; i < 2; ++i) {
+    g.tsf[i] = h_sf;
+    g.tsf_ld[i] = static_cast<int>(rows_all);
+    g.tsf_rows[i] = static_cast<int>(rows_all);
+  }
+  g.n_mblk = static_cast<int>(d / 128);
+  g.k_blocks = static_cast<int>(I / 128);
+  g.w_rows_per_group = static_cast<int>(d);
+  g.wsf_rb_per_group = static_cast<int>(d / 128);
+  g.up_offset = 0;
+  g.m_valid = static_cast<int>(d);
+  g.out = y;
+  g.ld_out = static_cast<int>(d);
+  g.out_sf = nullptr;
+  st = cuda_status(launch_gemm(g, s));
+  if (st != MOE_OK) return st;
+  if (ev) st = cuda_status(cudaEventRecord(ev[1], s));
+  return st;
+}
 
 // The two expert GEMMs over a chunk list already planned into the workspace.
 // seg 0: routed (a0 rows, w13_0 / w2_0 with G0 groups); seg 1: shared (a1 rows,
@@ -215,8 +326,8 @@ moe_status moe_route(const moe_config* cfg, const float* logits, const float* se
   if (cfg->T == 0) return MOE_OK;
   if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
   const float* bias = cfg->score == MOE_SCORE_SIGMOID_BIAS ? sel_bias : nullptr;
-  return cuda_status(launch_route(logits, bias, cfg->T, cfg->E, cfg->top_k, cfg->score, topk_idx,
-                                  topk_w, stream));
+  return cuda_status(launch_route(logits, 1, 0, bias, cfg->T, cfg->E, cfg->top_k, cfg->score,
+                                  topk_idx, topk_w, stream));
 }
 
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
@@ -231,9 +342,12 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
   const Layout L(*cfg);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  const int elem = cfg->act == MOE_F32 ? 4 : 2;
+  const bool fp8 = cfg->act == MOE_E4M3;
+  if (fp8 && cfg->T > 0 && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
+  const int elem = cfg->act == MOE_F32 ? 4 : (fp8 ? 1 : 2);
   return cuda_status(launch_permute(topk_idx, cfg->T, cfg->E, cfg->top_k, x, cfg->d_model * elem,
-                                    nullptr, 0, x_perm, nullptr, perm_token, inv_perm,
+                                    fp8 ? x_scale : nullptr, fp8 ? cfg->d_model / 128 : 0, x_perm,
+                                    fp8 ? x_perm_scale : nullptr, perm_token, inv_perm,
                                     group_offsets, at<int32_t>(ws, L.chunk_counts),
                                     at<unsigned>(ws, kHdrPermuteDone * sizeof(int)),
                                     status_word(ws), stream));
@@ -274,8 +388,31 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
     w13_b = at<void>(ws, L.w13_bf16);
     w2_b = at<void>(ws, L.w2_bf16);
   }
-  st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, at<Chunk>(ws, L.chunks),
-                               at<int32_t>(ws, kHdrNChunks * sizeof(int)), status_word(ws), stream));
+  if (cfg->act == MOE_E4M3) {
+    if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
+    if (n_groups > cfg->E + cfg->n_shared) return MOE_ERR_UNSUPPORTED;
+    uint32_t* a_sf = at<uint32_t>(ws, L.a_sf);
+    uint4* wsf13 = at<uint4>(ws, L.wsf13);
+    uint4* wsf2 = at<uint4>(ws, L.wsf2);
+    st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(a), a_scale, n_rows,
+                                         static_cast<int>(d), nullptr, a_sf, stream));
+    if (st == MOE_OK)
+      st = cuda_status(launch_weight_sf(w13_s, static_cast<size_t>(n_groups) * (2 * I / 128) * (d / 128),
+                                        wsf13, stream));
+    if (st == MOE_OK)
+      st = cuda_status(launch_weight_sf(w2_s, static_cast<size_t>(n_groups) * (d / 128) * (I / 128),
+                                        wsf2, stream));
+    if (st == MOE_OK)
+      st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRowsFP8,
+                                   at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                                   status_word(ws), stream));
+    if (st != MOE_OK) return st;
+    return run_ffn_fp8(*cfg, L, ws, a, a_sf, n_rows, w13, w2, wsf13, wsf2, n_groups, nullptr,
+                       nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0, n_rows, y, stream);
+  }
+  st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRows,
+                               at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                               status_word(ws), stream));
   if (st != MOE_OK) return st;
   return run_ffn(*cfg, L, ws, a_b, n_rows, w13_b, w2_b, n_groups, nullptr, 0, nullptr, nullptr, 0,
                  n_rows, y, stream);
@@ -305,7 +442,6 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
                               const float* x_scale, void* y, int32_t* topk_idx_out,
                               float* topk_w_out, void* ws, size_t ws_bytes, cudaStream_t stream,
                               cudaEvent_t* ev) {
-  (void)x_scale;
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (!wts || !ws) return MOE_ERR_INVALID_ARG;
@@ -315,6 +451,10 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if (c.n_shared > 0 && (!wts->ws13 || !wts->ws2)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y) || !aligned16(wts->wr) || !aligned16(wts->w13) ||
       !aligned16(wts->w2) || !aligned16(wts->ws13) || !aligned16(wts->ws2))
+    return MOE_ERR_INVALID_ARG;
+  const bool fp8 = c.act == MOE_E4M3;
+  if (fp8 && (!x_scale || !wts->w13_s || !wts->w2_s ||
+              (c.n_shared > 0 && (!wts->ws13_s || !wts->ws2_s))))
     return MOE_ERR_INVALID_ARG;
   const Layout L(c);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -351,6 +491,23 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
     ws13_b = at<char>(ws, L.w13_bf16) + 2 * E * 2 * I * d;
     ws2_b = at<char>(ws, L.w2_bf16) + 2 * E * d * I;
   }
+  // FP8 family: bf16 copy of x for the router (exact) and UE8M0 scale factors
+  const void* x_router = x_b;
+  uint32_t* x_sf = at<uint32_t>(ws, L.x_sf);
+  uint4* wsf13 = at<uint4>(ws, L.wsf13);
+  uint4* wsf2 = at<uint4>(ws, L.wsf2);
+  if (fp8) {
+    st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(x), x_scale, c.T,
+                                         static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf, s));
+    const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
+    const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
+    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w13_s, E * n13, wsf13, s));
+    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w2_s, E * n2, wsf2, s));
+    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws13_s, S * n13, wsf13 + E * n13, s));
+    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws2_s, S * n2, wsf2 + E * n2, s));
+    if (st != MOE_OK) return st;
+    x_router = at<void>(ws, L.x_bf16);
+  }
 
   // 1. router GEMM: logits[T, E] = x Wr^T (fp32)
   float* logits = at<float>(ws, L.logits);
@@ -358,13 +515,15 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   {
     GemmLaunch g{};
     g.mode = kRouter;
-    if (!make_tmap_bf16(&g.wmap[0], wr_b, E, d, 128) || !make_tmap_bf16(&g.tmap[0], x_b, T, d, 16))
+    if (!make_tmap_bf16(&g.wmap[0], wr_b, E, d, 128) || !make_tmap_bf16(&g.tmap[0], x_router, T, d, 16))
       return MOE_ERR_CUDA;
     g.wmap[1] = g.wmap[0];
     g.tmap[1] = g.tmap[0];
     g.router_T = static_cast<int>(T);
     g.n_mblk = static_cast<int>((E + 127) / 128);
     g.k_blocks = static_cast<int>(d / 64);
+    g.k_splits = router_splits(T, E, d);
+    g.split_stride = static_cast<long long>(T) * E;
     g.m_valid = static_cast<int>(E);
     g.out = logits;
     g.ld_out = static_cast<int>(E);
@@ -379,31 +538,45 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
   float* gate = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
   const float* bias = c.score == MOE_SCORE_SIGMOID_BIAS ? wts->sel_bias : nullptr;
-  st = cuda_status(launch_route(logits, bias, c.T, c.E, c.top_k, c.score, idx, gate, s));
+  st = cuda_status(launch_route(logits, router_splits(T, E, d), static_cast<long long>(T) * E, bias,
+                                c.T, c.E, c.top_k, c.score, idx, gate, s));
   if (st != MOE_OK) return st;
   if ((st = mark(2)) != MOE_OK) return st;
 
-  // 3. permute (bf16 rows)
+  // 3. permute (bf16 rows, or e4m3 rows + their scale factors)
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm_token = at<int32_t>(ws, L.perm_token);
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   void* x_perm = at<void>(ws, L.x_perm);
-  st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(d * 2), nullptr, 0,
-                                  x_perm, nullptr, perm_token, inv_perm, offsets,
+  uint32_t* x_perm_sf = at<uint32_t>(ws, L.x_perm_sf);
+  st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(fp8 ? d : d * 2),
+                                  nullptr, 0, x_perm, nullptr, perm_token, inv_perm, offsets,
                                   at<int32_t>(ws, L.chunk_counts),
                                   at<unsigned>(ws, kHdrPermuteDone * sizeof(int)), status, s));
+  if (st == MOE_OK && fp8)
+    st = cuda_status(launch_gather_sf(x_sf, c.T, static_cast<int>(d / 128), perm_token, offsets + E,
+                                      static_cast<int>(R), x_perm_sf, s));
   if (st != MOE_OK) return st;
   if ((st = mark(3)) != MOE_OK) return st;
 
   // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs
   st = cuda_status(launch_plan(offsets, c.E, static_cast<int>(R), c.n_shared, c.T,
-                               static_cast<int>(R), at<Chunk>(ws, L.chunks),
-                               at<int32_t>(ws, kHdrNChunks * sizeof(int)), status, s));
+                               static_cast<int>(R), fp8 ? kChunkRowsFP8 : kChunkRows,
+                               at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                               status, s));
   if (st != MOE_OK) return st;
   if ((st = mark(4)) != MOE_OK) return st;
   void* y_rows = at<void>(ws, L.y_rows);
-  st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows, s,
-               ev ? ev + 5 : nullptr);
+  if (fp8) {
+    const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
+    const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
+    st = run_ffn_fp8(c, L, ws, x_perm, x_perm_sf, R, w13_b, w2_b, wsf13, wsf2, E, x_b, x_sf, T, ws13_b,
+                     ws2_b, wsf13 + E * n13, wsf2 + E * n2, S, L.rows_all, y_rows, s,
+                     ev ? ev + 5 : nullptr);
+  } else {
+    st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows,
+                 s, ev ? ev + 5 : nullptr);
+  }
   if (st != MOE_OK) return st;
 
   // 7. combine

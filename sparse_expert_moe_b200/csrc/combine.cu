@@ -4,11 +4,11 @@
 //
 //   out[t] = sum_j w[t, j] * y_perm[inv_perm[t, j]] + sum_s y_shared_s[t]
 //
-// One CTA per token; each thread owns 8 consecutive columns (one 16-byte bf16
-// vector) and accumulates the k gathered rows in slot order in fp32 registers,
-// then the shared rows, then rounds once.  No atomics: every output element has
-// exactly one writer, so repeated runs are bit-identical.  HBM-bound: reads
-// (k + S) rows and writes one row per token.
+// One CTA per (token, 1024-column slice); each thread owns 8 consecutive columns
+// (one 16-byte bf16 vector) and accumulates the k gathered rows in slot order in
+// fp32 registers, then the shared rows, then rounds once.  No atomics: every
+// output element has exactly one writer, so repeated runs are bit-identical.
+// HBM-bound: reads (k + S) rows and writes one row per token.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint4* __restrict__ 
                                                       bool out_f32, void* __restrict__ out) {
   const int t = blockIdx.x;
   const int vec = d / 8;
+  const int v = blockIdx.y * blockDim.x + threadIdx.x;
   __shared__ int32_t rows[KMAX];
   __shared__ float ws[KMAX];
   if (threadIdx.x < k) {
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint4* __restrict__ 
     ws[threadIdx.x] = topk_w[static_cast<size_t>(t) * k + threadIdx.x];
   }
   __syncthreads();
-  for (int v = threadIdx.x; v < vec; v += blockDim.x) {
+  if (v < vec) {
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -90,10 +91,11 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, const fl
   const uint4* yp = static_cast<const uint4*>(y_perm);
   const uint4* ys = static_cast<const uint4*>(y_shared);
   if (!y_shared) n_shared = 0;
+  const dim3 grid(T, (d / 8 + 127) / 128);
   if (k <= 8)
-    combine_kernel<8><<<T, 128, 0, s>>>(yp, inv_perm, topk_w, ys, n_shared, T, d, k, R, out_f32, y);
+    combine_kernel<8><<<grid, 128, 0, s>>>(yp, inv_perm, topk_w, ys, n_shared, T, d, k, R, out_f32, y);
   else
-    combine_kernel<16><<<T, 128, 0, s>>>(yp, inv_perm, topk_w, ys, n_shared, T, d, k, R, out_f32, y);
+    combine_kernel<16><<<grid, 128, 0, s>>>(yp, inv_perm, topk_w, ys, n_shared, T, d, k, R, out_f32, y);
   return cudaGetLastError();
 }
 

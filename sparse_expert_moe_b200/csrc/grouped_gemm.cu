@@ -32,6 +32,7 @@
 // Chunks come from the planner below, largest groups first.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -40,13 +41,11 @@ namespace moe {
 namespace {
 
 constexpr int kBM = 128;                  // weight rows per tile (UMMA M)
-constexpr int kBK = 64;                   // K elements per stage (128 bytes of bf16)
-constexpr int kNT = kChunkRows;           // token rows per tile (UMMA N max)
+constexpr int kRowBytes = 128;            // K bytes per stage and row: one 128-byte swizzle row
 constexpr int kTokBox = 16;               // token rows per TMA box
-constexpr uint32_t kABytes = kBM * kBK * 2;
-constexpr uint32_t kBBytes = kNT * kBK * 2;
-constexpr uint32_t kTokBoxBytes = kTokBox * kBK * 2;
-constexpr int kThreads = 192;
+constexpr uint32_t kABytes = kBM * kRowBytes;
+constexpr uint32_t kTokBoxBytes = kTokBox * kRowBytes;
+constexpr uint32_t kSFAtomBytes = 512;    // 128 rows x 4 UE8M0 bytes (tcgen05.cp 32x128b source)
 
 struct DevParams {
   CUtensorMap wmap[2];
@@ -56,37 +55,87 @@ struct DevParams {
   int router_T;
   int n_mblk;
   int k_blocks;
+  int k_splits;               // router: K split across CTAs (partial outputs, summed later)
+  int k_per_split;            // k blocks per split
+  long long split_stride;     // elements between the partial outputs of consecutive splits
   int w_rows_per_group;
   int up_offset;
   int m_valid;
   void* out;
   int ld_out;
   int* status;
+  // FP8 block scaling
+  const uint4* wsf[2];        // [groups][row blocks][k blocks] UE8M0 x16 per 128x128 weight block
+  int wsf_rb_per_group;       // 128-row blocks of the weight matrix per group
+  const uint32_t* tsf[2];     // [k blocks][rows] UE8M0 x4 per (128-element block, token row)
+  int tsf_ld[2];
+  int tsf_rows[2];
+  uint32_t* out_sf;           // FFN1 (FP8): [I / 128][rows] scales of the requantised h
+  int ld_out_sf;
 };
 
+template <int MODE>
+struct Cfg {
+  static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8;
+  static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8;   // gate + up accumulators
+  static constexpr int kATiles = kGLU ? 2 : 1;
+  static constexpr int kNT = kFP8 ? kChunkRowsFP8 : kChunkRows;     // max tokens per tile
+  static constexpr uint32_t kBBytes = kNT * kRowBytes;
+  static constexpr uint32_t kSFBytes = kFP8 ? (kATiles + 1) * kSFAtomBytes : 0;
+  static constexpr uint32_t kStageBytes =
+      ((kATiles * kABytes + kBBytes + kSFBytes + 1023) / 1024) * 1024;
+  static constexpr int kStages = kGLU ? 4 : 6;
+  static constexpr uint32_t kAccCols = kGLU ? 2 * kNT : kNT;        // per accumulator buffer
+  static constexpr uint32_t kSFColsPerStage = 16;                     // <= 3 atoms x 4 columns
+  static constexpr uint32_t kSFCols = kFP8 ? kStages * kSFColsPerStage : 0;
+  static constexpr uint32_t kColsUsed = 2 * kAccCols + kSFCols;
+  static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256 : 512;
+  static constexpr int kThreads = kFP8 ? 224 : 192;                 // + one scale-factor warp
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
+  static_assert(kColsUsed <= 512, "TMEM budget");
+};
+
+template <int MODE>
 __device__ __forceinline__ Chunk get_chunk(const DevParams& p, int ci) {
   if (p.chunks) return p.chunks[ci];
   Chunk c;
   c.seg = 0;
   c.group = 0;
-  c.b_row = ci * kNT;
+  c.b_row = ci * Cfg<MODE>::kNT;
   c.o_row = c.b_row;
-  c.nrows = min(kNT, p.router_T - c.b_row);
+  c.nrows = min(Cfg<MODE>::kNT, p.router_T - c.b_row);
   return c;
 }
 
-template <int MODE>
-struct Cfg {
-  static constexpr int kATiles = MODE == kFFN1 ? 2 : 1;
-  static constexpr uint32_t kStageBytes = kATiles * kABytes + kBBytes;
-  static constexpr int kStages = MODE == kFFN1 ? 4 : 6;
-  static constexpr uint32_t kAccCols = MODE == kFFN1 ? 2 * kNT : kNT;   // per buffer
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;                  // 512 or 256
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
+// Tile t -> (chunk, weight block, K split).  Splits are fastest, then weight blocks.
+struct TileCoord {
+  int chunk, mb, split, kb0, kb1;
 };
+__device__ __forceinline__ TileCoord tile_coord(const DevParams& p, int t) {
+  TileCoord tc;
+  tc.split = t % p.k_splits;
+  const int r = t / p.k_splits;
+  tc.chunk = r / p.n_mblk;
+  tc.mb = r % p.n_mblk;
+  tc.kb0 = tc.split * p.k_per_split;
+  tc.kb1 = min(p.k_blocks, tc.kb0 + p.k_per_split);
+  return tc;
+}
+
+// Smallest e with amax <= 448 * 2^e (amax as fp32 bits, non-negative), clamped to the
+// UE8M0 range: the power-of-two scale of an e4m3 block.  448 = 1.75 * 2^8, so with
+// amax = m * 2^ea (m in [1, 2)): e = ea - 8 when m <= 1.75, else ea - 7.
+__device__ __forceinline__ int e4m3_scale_exponent(uint32_t amax_bits) {
+  if (amax_bits == 0) return 0;
+  const int ea = static_cast<int>((amax_bits >> 23) & 0xFFu);
+  if (ea == 0) return -127;
+  const int e = (ea - 127) - ((amax_bits & 0x7FFFFFu) <= 0x600000u ? 8 : 7);
+  return max(-127, min(127, e));
+}
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ DevParams p) {
+__global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ DevParams p) {
   using C = Cfg<MODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -96,20 +145,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* tfull_bar = empty_bar + C::kStages;
   uint64_t* tempty_bar = tfull_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  uint64_t* red_bar = tempty_bar + 2;                            // [2] FP8 amax exchange
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* red = reinterpret_cast<uint32_t*>(tmem_slot + 4);   // [2][4][16] FP8 amax exchange
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&full_bar[i], 1);
+      mbar_init(&full_bar[i], C::kFP8 ? 1 + 32 : 1);
       mbar_init(&empty_bar[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
       mbar_init(&tempty_bar[i], 128);
+      mbar_init(&red_bar[i], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -125,36 +177,38 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_chunks = p.chunks ? *p.n_chunks : (p.router_T + kNT - 1) / kNT;
-  const int n_tiles = n_chunks * p.n_mblk;
+  const int n_chunks = p.chunks ? *p.n_chunks : (p.router_T + C::kNT - 1) / C::kNT;
+  const int n_tiles = n_chunks * p.n_mblk * p.k_splits;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const Chunk c = get_chunk(p, t / p.n_mblk);
-        const int mb = t % p.n_mblk;
+        const TileCoord tc = tile_coord(p, t);
+        const Chunk c = get_chunk<MODE>(p, tc.chunk);
+        const int mb = tc.mb;
         const int a_row = c.group * p.w_rows_per_group + mb * kBM;
         const int nbox = (c.nrows + kTokBox - 1) / kTokBox;
-        // FFN2 reads the h rows FFN1 wrote (output numbering); the others read b_row
-        const int tok_row = MODE == kFFN2 ? c.o_row : c.b_row;
+        // the second GEMM reads the h rows the first one wrote (output numbering)
+        const int tok_row = (MODE == kFFN2 || MODE == kFFN2F8) ? c.o_row : c.b_row;
         const uint32_t bytes = C::kATiles * kABytes + nbox * kTokBoxBytes;
         const CUtensorMap* wm = &p.wmap[c.seg];
         const CUtensorMap* tm = &p.tmap[c.seg];
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
           uint8_t* st = tiles + stage * C::kStageBytes;
+          const int kx = kb * (C::kFP8 ? 128 : 64);   // element coordinate of this K block
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          tma_load_2d(st, wm, &full_bar[stage], kb * kBK, a_row);
-          if (MODE == kFFN1) tma_load_2d(st + kABytes, wm, &full_bar[stage], kb * kBK, a_row + p.up_offset);
+          tma_load_2d(st, wm, &full_bar[stage], kx, a_row);
+          if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[stage], kx, a_row + p.up_offset);
           uint8_t* bt = st + C::kATiles * kABytes;
           for (int i = 0; i < nbox; ++i)
-            tma_load_2d(bt + i * kTokBoxBytes, tm, &full_bar[stage], kb * kBK, tok_row + i * kTokBox);
+            tma_load_2d(bt + i * kTokBoxBytes, tm, &full_bar[stage], kx, tok_row + i * kTokBox);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
@@ -170,16 +224,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       bool ok = true;
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const Chunk c = get_chunk(p, t / p.n_mblk);
+        const TileCoord tc = tile_coord(p, t);
+        const Chunk c = get_chunk<MODE>(p, tc.chunk);
         const int n_pad = (c.nrows + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(kBM, n_pad);
+        const uint32_t idesc = C::kFP8 ? idesc_e4m3_bs(kBM, n_pad) : idesc_bf16_f32(kBM, n_pad);
         const uint32_t acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
-        const uint32_t d1 = d0 + kNT;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        const uint32_t d1 = d0 + C::kNT;
+        for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) {
             ok = false;
             break;
@@ -187,12 +242,32 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           tc_fence_after();
           const uint32_t st = smem_u32(tiles + stage * C::kStageBytes);
           const uint32_t bt = st + C::kATiles * kABytes;
+          if (C::kFP8) {
+            // scale factors of this stage: smem (written by the scale warp) -> TMEM
+            fence_proxy_async_smem();
+            const uint32_t sf_smem = bt + C::kBBytes;
+            const uint32_t sfa = tmem_base + 2 * C::kAccCols + stage * C::kSFColsPerStage;
+            const uint32_t sfb = sfa + C::kATiles * 4;
+            tmem_cp_32x128b_warpx4(sfa, smem_desc_noswizzle(sf_smem));
+            if (C::kGLU) tmem_cp_32x128b_warpx4(sfa + 4, smem_desc_noswizzle(sf_smem + kSFAtomBytes));
+            tmem_cp_32x128b_warpx4(sfb, smem_desc_noswizzle(sf_smem + C::kATiles * kSFAtomBytes));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t accum = (kb | kk) ? 1u : 0u;
-            const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
-            umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, accum);
-            if (MODE == kFFN1) umma_bf16(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, accum);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
+              const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
+              umma_e4m3_bs(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, sfa, sfb, accum);
+              if (C::kGLU)
+                umma_e4m3_bs(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, sfa + 4, sfb,
+                             accum);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
+              const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
+              umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, accum);
+              if (C::kGLU) umma_bf16(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, accum);
+            }
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == C::kStages) {
@@ -204,14 +279,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int sub = warp & 3;                 // TMEM lane quadrant of this warp
     const int m_local = sub * 32 + lane;      // weight row inside the tile
     int it = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-      const Chunk c = get_chunk(p, t / p.n_mblk);
-      const int mb = t % p.n_mblk;
+    uint32_t rbuf = 0, rpar = 0;              // FP8 amax exchange: buffer and per-buffer parity bits
+    bool epi_ok = true;
+    for (int t = blockIdx.x; t < n_tiles && epi_ok; t += gridDim.x, ++it) {
+      const TileCoord tc = tile_coord(p, t);
+      const Chunk c = get_chunk<MODE>(p, tc.chunk);
+      const int mb = tc.mb;
       const uint32_t acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status);
@@ -222,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       for (int n0 = 0; n0 < c.nrows; n0 += 16) {
         if (MODE == kFFN1) {
           float g[16], u[16];
-          tmem_ld16x2(tb + n0, tb + kNT + n0, g, u);
+          tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
           __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -231,7 +309,43 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               h[static_cast<size_t>(c.o_row + n0 + i) * p.ld_out + m] = __float2bfloat16_rn(s * u[i]);
             }
           }
-        } else if (MODE == kFFN2) {
+        } else if (MODE == kFFN1F8) {
+          // SwiGLU, then requantise h to e4m3 with one power-of-two scale per token per
+          // 128 h columns (this tile's columns): amax across the tile's 128 threads, the
+          // four warps' partial maxima exchanged through shared memory (double-buffered,
+          // one mbarrier per buffer, bounded waits)
+          float g[16], u[16], hv[16];
+          tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            hv[i] = g[i] / (1.0f + __expf(-g[i])) * u[i];
+            const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[i])));
+            if (lane == 0) red[(rbuf * 4 + sub) * 16 + i] = wmax;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&red_bar[rbuf]);
+          const bool rok = mbar_wait(&red_bar[rbuf], (rpar >> rbuf) & 1u, abort_flag, p.status);
+          rpar ^= 1u << rbuf;
+          if (!__all_sync(0xffffffffu, rok)) {
+            epi_ok = false;
+            break;
+          }
+          uint8_t* h = static_cast<uint8_t*>(p.out);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t* r = red + rbuf * 64 + i;
+            const uint32_t amax = max(max(r[0], r[16]), max(r[32], r[48]));
+            const int e = e4m3_scale_exponent(amax);
+            if (n0 + i < c.nrows) {
+              const __nv_fp8_storage_t q = __nv_cvt_float_to_fp8(scalbnf(hv[i], -e), __NV_SATFINITE, __NV_E4M3);
+              h[static_cast<size_t>(c.o_row + n0 + i) * p.ld_out + m] = q;
+              if (m_local == 0)
+                p.out_sf[static_cast<size_t>(mb) * p.ld_out_sf + c.o_row + n0 + i] =
+                    0x01010101u * static_cast<uint32_t>(e + 127);
+            }
+          }
+          rbuf ^= 1u;
+        } else if (MODE == kFFN2 || MODE == kFFN2F8) {
           float v[16];
           tmem_ld16(tb + n0, v);
           __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.out);
@@ -242,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         } else {
           float v[16];
           tmem_ld16(tb + n0, v);
-          float* lg = static_cast<float*>(p.out);
+          float* lg = static_cast<float*>(p.out) + tc.split * p.split_stride;
           if (m < p.m_valid) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -253,6 +367,51 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
     }
+  } else if (C::kFP8) {
+    // ------------------------------------------------------------ scale-factor warp (FP8)
+    // Per stage: the 512-byte scale atoms of the weight tile(s) (one UE8M0 value for the
+    // whole 128x128 block, replicated) and of the token rows (row n's 4 bytes at
+    // (n % 32) * 16 + (n / 32) * 4), copied with cp.async; each lane's completion
+    // arrives on the stage's full barrier.
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    const int up_rb = p.up_offset / kBM;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord(p, t);
+      const Chunk c = get_chunk<MODE>(p, tc.chunk);
+      const int mb = tc.mb;
+      const int n_pad = (c.nrows + 15) & ~15;
+      const int tok_row = MODE == kFFN2F8 ? c.o_row : c.b_row;
+      const uint4* wsf = p.wsf[c.seg] + static_cast<size_t>(c.group) * p.wsf_rb_per_group * p.k_blocks;
+      const uint32_t* tsf = p.tsf[c.seg];
+      const int tld = p.tsf_ld[c.seg], trows = p.tsf_rows[c.seg];
+      for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
+        const bool w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sf = tiles + stage * C::kStageBytes + C::kATiles * kABytes + C::kBBytes;
+        cp_async_16(sf + lane * 16, wsf + static_cast<size_t>(mb) * p.k_blocks + kb);
+        if (C::kGLU)
+          cp_async_16(sf + kSFAtomBytes + lane * 16, wsf + static_cast<size_t>(up_rb + mb) * p.k_blocks + kb);
+        uint8_t* sfb = sf + C::kATiles * kSFAtomBytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int n = lane + 32 * j;
+          if (n < n_pad) {
+            const int row = min(tok_row + n, trows - 1);
+            cp_async_4(sfb + lane * 16 + j * 4, tsf + static_cast<size_t>(kb) * tld + row);
+          }
+        }
+        cp_async_mbar_arrive_noinc(&full_bar[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -264,10 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 // ---------------------------------------------------------------- planner
 // One CTA.  Validates the offsets, orders the groups by size (largest first,
 // ties by index: routed before shared), splits each into chunks of at most
-// kChunkRows rows and writes the chunk list and its length.
+// `cr` rows (the GEMM's token tile) and writes the chunk list and its length.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ offsets, int G,
                                                     int n_rows, int n_shared, int T,
-                                                    int shared_o_row, Chunk* __restrict__ chunks,
+                                                    int shared_o_row, int cr,
+                                                    Chunk* __restrict__ chunks,
                                                     int32_t* __restrict__ n_chunks, int* status) {
   __shared__ int32_t sz[kMaxGroups];
   __shared__ int32_t start[kMaxGroups];
@@ -314,8 +474,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   // exclusive scan of chunk counts in rank order; thread owns ranks 2*tid, 2*tid+1
   int c0 = 0, c1 = 0;
   const int r0 = 2 * tid, r1 = 2 * tid + 1;
-  if (r0 < NG) c0 = (sz[order[r0]] + kChunkRows - 1) / kChunkRows;
-  if (r1 < NG) c1 = (sz[order[r1]] + kChunkRows - 1) / kChunkRows;
+  if (r0 < NG) c0 = (sz[order[r0]] + cr - 1) / cr;
+  if (r1 < NG) c1 = (sz[order[r1]] + cr - 1) / cr;
   const int local = c0 + c1;
   const int lane = tid & 31, warp = tid >> 5;
   int incl = local;
@@ -337,13 +497,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     const int s = sz[g];
     const bool shared = g >= G;
     int base = cbase[r];
-    for (int c = 0; c * kChunkRows < s; ++c) {
+    for (int c = 0; c * cr < s; ++c) {
       Chunk ch;
       ch.seg = shared ? 1 : 0;
       ch.group = shared ? g - G : g;
-      ch.b_row = start[g] + c * kChunkRows;
-      ch.o_row = shared ? shared_o_row + (g - G) * T + c * kChunkRows : ch.b_row;
-      ch.nrows = min(kChunkRows, s - c * kChunkRows);
+      ch.b_row = start[g] + c * cr;
+      ch.o_row = shared ? shared_o_row + (g - G) * T + c * cr : ch.b_row;
+      ch.nrows = min(cr, s - c * cr);
       ch.pad0 = ch.pad1 = ch.pad2 = 0;
       chunks[base + c] = ch;
     }
@@ -354,10 +514,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 }  // namespace
 
 cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared, int T,
-                        int shared_o_row, Chunk* chunks, int32_t* n_chunks, int* status,
-                        cudaStream_t s) {
-  plan_kernel<<<1, 1024, 0, s>>>(offsets, G, n_rows, n_shared, T, shared_o_row, chunks, n_chunks,
-                                 status);
+                        int shared_o_row, int chunk_rows, Chunk* chunks, int32_t* n_chunks,
+                        int* status, cudaStream_t s) {
+  plan_kernel<<<1, 1024, 0, s>>>(offsets, G, n_rows, n_shared, T, shared_o_row, chunk_rows, chunks,
+                                 n_chunks, status);
   return cudaGetLastError();
 }
 
@@ -375,23 +535,35 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   p.router_T = g.router_T;
   p.n_mblk = g.n_mblk;
   p.k_blocks = g.k_blocks;
+  p.k_splits = g.k_splits > 1 ? g.k_splits : 1;
+  p.k_per_split = (g.k_blocks + p.k_splits - 1) / p.k_splits;
+  p.split_stride = g.split_stride;
   p.w_rows_per_group = g.w_rows_per_group;
   p.up_offset = g.up_offset;
   p.m_valid = g.m_valid;
   p.out = g.out;
   p.ld_out = g.ld_out;
   p.status = g.status;
+  for (int i = 0; i < 2; ++i) {
+    p.wsf[i] = g.wsf[i];
+    p.tsf[i] = g.tsf[i];
+    p.tsf_ld[i] = g.tsf_ld[i];
+    p.tsf_rows[i] = g.tsf_rows[i];
+  }
+  p.wsf_rb_per_group = g.wsf_rb_per_group;
+  p.out_sf = g.out_sf;
+  p.ld_out_sf = g.ld_out_sf;
   cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::kSmemBytes));
   if (err != cudaSuccess) return err;
   int grid = g.num_sms;
   if (MODE == kRouter) {
-    const int tiles = ((g.router_T + kNT - 1) / kNT) * g.n_mblk;
+    const int tiles = ((g.router_T + C::kNT - 1) / C::kNT) * g.n_mblk * p.k_splits;
     if (tiles < grid) grid = tiles;
     if (grid == 0) return cudaSuccess;
   }
-  grouped_gemm_kernel<MODE><<<grid, kThreads, C::kSmemBytes, s>>>(p);
+  grouped_gemm_kernel<MODE><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -400,6 +572,8 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
     case kRouter: return launch_mode<kRouter>(g, s);
     case kFFN1: return launch_mode<kFFN1>(g, s);
     case kFFN2: return launch_mode<kFFN2>(g, s);
+    case kFFN1F8: return launch_mode<kFFN1F8>(g, s);
+    case kFFN2F8: return launch_mode<kFFN2F8>(g, s);
     default: return cudaErrorInvalidValue;
   }
 }

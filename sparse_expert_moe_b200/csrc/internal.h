@@ -24,17 +24,34 @@ struct Chunk {
   int32_t seg, group, b_row, o_row, nrows, pad0, pad1, pad2;
 };
 
-constexpr int kChunkRows = 128;   // tokens per GEMM tile (UMMA N <= 128)
+constexpr int kChunkRows = 128;     // tokens per GEMM tile, bf16 (UMMA N <= 128)
+constexpr int kChunkRowsFP8 = 112;  // tokens per GEMM tile, FP8 (TMEM also holds scale factors)
 constexpr int kMaxGroups = 1024 + 8;
 
 // Upper bound on the chunks of `rows` rows spread over `groups` groups.
-inline int64_t max_chunks(int64_t rows, int64_t groups) {
-  return rows / kChunkRows + groups + 1;
+inline int64_t max_chunks(int64_t rows, int64_t groups, int chunk_rows = kChunkRowsFP8) {
+  return rows / chunk_rows + groups + 1;
 }
 
 // ---------------------------------------------------------------- kernels
-cudaError_t launch_route(const float* logits, const float* sel_bias, int T, int E, int k,
-                         int score, int32_t* topk_idx, float* topk_w, cudaStream_t s);
+// logits: n_partials partial [T, E] arrays `partial_stride` floats apart, summed in
+// order before scoring (1 = plain logits).
+cudaError_t launch_route(const float* logits, int n_partials, long long partial_stride,
+                         const float* sel_bias, int T, int E, int k, int score, int32_t* topk_idx,
+                         float* topk_w, cudaStream_t s);
+
+// K splits of the router GEMM for T tokens, E experts and d_model: enough CTAs to
+// cover the 148 SMs when the (token chunk, expert block) tiles alone cannot;
+// every split non-empty.  Host only.
+inline int router_splits(int64_t T, int64_t E, int64_t d) {
+  const int64_t tiles = ((T + 127) / 128) * ((E + 127) / 128);
+  const int64_t kb = d / 64;
+  int64_t s = tiles >= 148 ? 1 : 148 / tiles;
+  if (s > kb) s = kb;
+  if (s < 1) s = 1;
+  const int64_t per = (kb + s - 1) / s;
+  return static_cast<int>((kb + per - 1) / per);
+}
 
 // Permutation.  `chunk_counts` holds ceil(T / 256) * E ints; `done` one zeroed
 // counter (left zero on exit).
@@ -49,10 +66,10 @@ inline int permute_chunks(int T) { return (T + 255) / 256; }
 // by n_shared groups of T rows each (token rows 0..T-1 of the unpermuted
 // activations, output rows shared_o_row + s*T).  Heavy groups first.
 cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared, int T,
-                        int shared_o_row, Chunk* chunks, int32_t* n_chunks, int* status,
-                        cudaStream_t s);
+                        int shared_o_row, int chunk_rows, Chunk* chunks, int32_t* n_chunks,
+                        int* status, cudaStream_t s);
 
-enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2 };
+enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4 };
 
 struct GemmLaunch {
   int mode;
@@ -63,7 +80,9 @@ struct GemmLaunch {
   const int32_t* n_chunks;   // device (FFN modes)
   int router_T;              // router mode: tokens
   int n_mblk;                // 128-row weight blocks per group
-  int k_blocks;              // K / 64
+  int k_blocks;              // K / 64 (bf16) or K / 128 (e4m3)
+  int k_splits;              // router: K split across CTAs (1 = none); every split non-empty
+  long long split_stride;    // router: elements between consecutive partial outputs
   int w_rows_per_group;      // weight rows per group (FFN1: 2I, FFN2: d)
   int up_offset;             // FFN1: I
   int m_valid;               // router: E
@@ -71,6 +90,16 @@ struct GemmLaunch {
   int ld_out;
   int* status;
   int num_sms;
+  // FP8 modes: weight block scales (UE8M0 replicated x16, [groups][row blocks][k blocks])
+  // and token scales (UE8M0 replicated x4, [k blocks][rows]) per segment; FFN1 writes
+  // the scales of its requantised output to out_sf ([I / 128][ld_out_sf]).
+  const uint4* wsf[2];
+  int wsf_rb_per_group;
+  const uint32_t* tsf[2];
+  int tsf_ld[2];
+  int tsf_rows[2];
+  uint32_t* out_sf;
+  int ld_out_sf;
 };
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s);
 
@@ -78,6 +107,20 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s);
 // {64 columns, box_rows rows}, 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+// Same for 1-byte (e4m3) elements, box {128 columns, box_rows rows}.
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows);
+
+// FP8 preparation kernels.
+// x e4m3 [T, d] + x_scale fp32 [T, d/128] -> x_bf16 [T, d] (exact) and x_sf [d/128][T]
+// (UE8M0 replicated x4).  Either output may be null.
+cudaError_t launch_act_prep_fp8(const uint8_t* x, const float* x_scale, int T, int d, void* x_bf16,
+                                uint32_t* x_sf, cudaStream_t s);
+// fp32 power-of-two block scales [n] -> UE8M0 replicated x16 [n] (uint4).
+cudaError_t launch_weight_sf(const float* scales, size_t n, uint4* out, cudaStream_t s);
+// x_perm_sf[kb][r] = x_sf[kb][perm_token[r]] for r < offsets_total (device).
+cudaError_t launch_gather_sf(const uint32_t* x_sf, int T, int kbs, const int32_t* perm_token,
+                             const int32_t* total, int R, uint32_t* x_perm_sf, cudaStream_t s);
 
 cudaError_t launch_combine(const void* y_perm, const int32_t* inv_perm, const float* topk_w,
                            const void* y_shared, int n_shared, int T, int d, int k, int R,

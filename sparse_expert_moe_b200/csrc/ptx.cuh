@@ -226,4 +226,75 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t taddr0, uint32_t taddr1, fl
   }
 }
 
+// ---------------------------------------------------------------- FP8 block scaling
+// Ampere-style asynchronous global->shared copies (4 or 16 bytes) and the mbarrier
+// arrival that fires when all of this thread's earlier cp.async copies complete
+// (.noinc: the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Orders this thread's view of shared memory between the generic proxy (plain and
+// cp.async writes) and the async proxy (TMA, tcgen05 reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory descriptor of a block of 8-row x 16-byte core matrices without
+// swizzle (rows 16 bytes apart, core matrices 128 bytes apart): the source
+// layout tcgen05.cp expects for a 32-row x 128-bit copy.
+__device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;   // leading byte offset (one 16-byte column: unused)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset: next 8-row core matrix
+  d |= static_cast<uint64_t>(1u) << 46;          // version
+  return d;                                     // layout type 0: no swizzle
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM columns taddr..taddr+3,
+// replicated into all four 32-lane sub-partitions (the scale-factor layout of a
+// 128-row operand: row r's bytes sit in lane r % 32, column r / 32).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: e4m3 A and B
+// (format 0), both K-major, UE8M0 scale factors (bit 23), shape M x N, scale
+// factor ids 0.
+__host__ __device__ constexpr uint32_t idesc_e4m3_bs(int M, int N) {
+  return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= (A * sfa) x (B * sfb)^T over K = 32 e4m3 elements, one scale per
+// row per 32 elements read from TMEM at sfa_tmem / sfb_tmem.
+__device__ __forceinline__ void umma_e4m3_bs(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Named barrier over `count` threads (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 }  // namespace moe

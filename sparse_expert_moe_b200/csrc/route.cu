@@ -6,10 +6,12 @@
 // bias routing" ("Chapter 7: Serving Mega MoE at scale").
 //
 // Each lane holds experts lane, lane+32, ... of the token's logit row (coalesced
-// 128-byte loads).  k rounds of a warp-wide arg-max (shuffle butterfly; key
-// descending, equal keys to the lower expert index) pick the slots in order;
-// lane j keeps slot j and computes its gate with one more butterfly.  HBM-bound:
-// the kernel reads T*E*4 bytes and writes T*k*8.
+// 128-byte loads); when the router GEMM split K across CTAs, the partial logits
+// are summed here in a fixed order, so repeated runs are bit-identical.  k rounds
+// of a warp-wide arg-max (shuffle butterfly; key descending, equal keys to the
+// lower expert index) pick the slots in order; lane j keeps slot j and computes
+// its gate with one more butterfly.  HBM-bound: the kernel reads
+// n_partials * T * E * 4 bytes and writes T * k * 8.
 #include <cfloat>
 #include <climits>
 #include <cuda_runtime.h>
@@ -26,7 +28,8 @@ __device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
 }
 
 template <int VPL>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int n_partials,
+                                                    long long partial_stride,
                                                     const float* __restrict__ sel_bias, int T, int E,
                                                     int k, int score, int32_t* __restrict__ topk_idx,
                                                     float* __restrict__ topk_w) {
@@ -42,6 +45,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     float l = 0.f, kk = -FLT_MAX;
     if (e < E) {
       l = __ldg(row + e);
+      for (int q = 1; q < n_partials; ++q) l += __ldg(row + q * partial_stride + e);
       if (score == 0) {
         kk = l;
       } else {
@@ -107,23 +111,30 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 
 }  // namespace
 
-cudaError_t launch_route(const float* logits, const float* sel_bias, int T, int E, int k, int score,
-                         int32_t* topk_idx, float* topk_w, cudaStream_t s) {
+cudaError_t launch_route(const float* logits, int n_partials, long long partial_stride,
+                         const float* sel_bias, int T, int E, int k, int score, int32_t* topk_idx,
+                         float* topk_w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int threads = 256;
   const int blocks = (T + 7) / 8;
   if (E <= 32)
-    route_kernel<1><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+    route_kernel<1><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
+                                               k, score, topk_idx, topk_w);
   else if (E <= 64)
-    route_kernel<2><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+    route_kernel<2><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
+                                               k, score, topk_idx, topk_w);
   else if (E <= 128)
-    route_kernel<4><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+    route_kernel<4><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
+                                               k, score, topk_idx, topk_w);
   else if (E <= 256)
-    route_kernel<8><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+    route_kernel<8><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
+                                               k, score, topk_idx, topk_w);
   else if (E <= 512)
-    route_kernel<16><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+    route_kernel<16><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
+                                               k, score, topk_idx, topk_w);
   else
-    route_kernel<32><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+    route_kernel<32><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
+                                               k, score, topk_idx, topk_w);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,113 @@
+"""The FP8 block-scaled path (e4m3 activations with 1x128 scales, e4m3 weights with
+128x128 scales, h requantised to e4m3 in the first GEMM's epilogue) against the fp64
+oracle on the decoded input values.  Bar: max relative error 6e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_expert_moe_b200 import inputs, moe
+
+from helpers import margin_workload, max_rel_err, oracle_layer
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL_FP8 = 6e-2
+
+
+def _e4m3(a, br, bc):
+    return inputs.to_e4m3_blocks(np.asarray(a, np.float32), br, bc)
+
+
+def _dq(q, s, br, bc):
+    return oracle.dequantize_blocks(q.view(torch.uint8).numpy(), s.numpy(), br, bc)
+
+
+@pytest.mark.parametrize("sizes,d,I", [
+    ([5, 0, 1, 130, 16, 17, 0, 112], 256, 256),
+    ([300], 128, 384),
+    ([1, 2, 3], 512, 128),
+])
+def test_grouped_ffn_fp8_vs_oracle(sizes, d, I):
+    rng = np.random.default_rng(sum(sizes) + d)
+    G, n_rows = len(sizes), sum(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    a, a_s = _e4m3(rng.standard_normal((n_rows, d)) * np.exp2(rng.integers(-3, 3, (n_rows, 1))), 1, 128)
+    w13 = [_e4m3(rng.standard_normal((2 * I, d)) * 0.05 * 2.0 ** rng.integers(-2, 3), 128, 128)
+           for _ in range(G)]
+    w2 = [_e4m3(rng.standard_normal((d, I)) * 0.05 * 2.0 ** rng.integers(-2, 3), 128, 128)
+          for _ in range(G)]
+    W13 = torch.stack([q for q, _ in w13]).to(DEV)
+    S13 = torch.stack([s for _, s in w13]).to(DEV)
+    W2 = torch.stack([q for q, _ in w2]).to(DEV)
+    S2 = torch.stack([s for _, s in w2]).to(DEV)
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0, act="e4m3", weight="e4m3")
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows, a.to(DEV), a_s.to(DEV),
+                        W13, S13, W2, S2, y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    av = _dq(a, a_s, 1, 128)
+    ref = np.zeros((n_rows, d))
+    for g in range(G):
+        lo, hi = offsets[g], offsets[g + 1]
+        if hi > lo:
+            ref[lo:hi] = oracle.swiglu_expert(av[lo:hi], _dq(*w13[g], 128, 128), _dq(*w2[g], 128, 128))
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert max_rel_err(got, ref) < TOL_FP8
+
+
+def test_permute_fp8_rows_and_scales():
+    T, E, k, d = 300, 32, 4, 256
+    rng = np.random.default_rng(9)
+    idx, _ = oracle.route(rng.uniform(-3, 3, (T, E)), "softmax", k)
+    x, xs = _e4m3(rng.standard_normal((T, d)), 1, 128)
+    cfg = moe.make_config(T, d, E, k, 128, 0, act="e4m3", weight="e4m3")
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    R = T * k
+    x_perm = torch.zeros((R, d), dtype=torch.uint8, device=DEV)
+    x_perm_s = torch.zeros((R, d // 128), dtype=torch.float32, device=DEV)
+    perm_token = torch.empty(R, dtype=torch.int32, device=DEV)
+    inv_perm = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    moe.moe_permute(cfg, torch.from_numpy(idx.astype(np.int32)).to(DEV), x.view(torch.uint8).to(DEV),
+                    xs.to(DEV), x_perm, x_perm_s, perm_token, inv_perm, offsets, ws)
+    ro, rp, ri = oracle.permute(idx, E)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(perm_token.cpu().numpy(), rp)
+    assert np.array_equal(inv_perm.cpu().numpy(), ri)
+    tp = torch.from_numpy(rp)
+    assert torch.equal(x_perm.cpu(), x.view(torch.uint8)[tp])
+    assert torch.equal(x_perm_s.cpu(), xs[tp])
+
+
+def _check_fp8_layer(wl, rows=None):
+    layer = moe.DeviceLayer.from_workload(wl, DEV)
+    idx = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.int32, device=DEV)
+    gw = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.float32, device=DEV)
+    y = layer.forward(wl.x.to(DEV), wl.x_scale.to(DEV), topk_idx=idx, topk_w=gw)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(layer.ws) == 0
+    got, idx, gw = y.float().cpu().numpy(), idx.cpu().numpy(), gw.cpu().numpy()
+    ref, r = oracle_layer(wl, rows=rows, return_routing=True)
+    if rows is not None:
+        got, idx, gw = got[rows], idx[rows], gw[rows]
+    assert np.array_equal(idx, r["idx"])
+    np.testing.assert_allclose(gw, r["gates"], rtol=1e-5, atol=1e-6)
+    err = max_rel_err(got, ref)
+    assert err < TOL_FP8, err
+
+
+@pytest.mark.parametrize("T,d,E,k,I,S", [(70, 256, 16, 4, 256, 1), (300, 384, 8, 2, 128, 2),
+                                         (1, 128, 4, 1, 128, 1)])
+def test_layer_fp8_custom(T, d, E, k, I, S):
+    spec = inputs.custom_spec(T, d, E, k, I, S, act="e4m3", weight="e4m3")
+    _check_fp8_layer(margin_workload(spec, seed=T + 1))
+
+
+@pytest.mark.slow
+def test_layer_fp8_full_size_sampled():
+    wl = inputs.load_workload("r1_prefill_fp8")
+    rows = np.sort(np.random.default_rng(1).choice(wl.spec.T, 12, replace=False))
+    _check_fp8_layer(wl, rows=rows)
