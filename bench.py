@@ -178,6 +178,26 @@ def read_traffic(kernel_key):
 
 
 # ---------------------------------------------------------------------------
+# replicas: one layer copy per rank, timed together
+# ---------------------------------------------------------------------------
+
+def max_over_ranks_dist(v, world, device):
+    """Max of a per-rank value over all ranks (the slowest replica sets the time)."""
+    if world == 1:
+        return float(v)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank, world, ms_total_max, steps):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (ms_total_max * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # the reference arm: the fp64 oracle on the host
 # ---------------------------------------------------------------------------
 
@@ -338,11 +358,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_dist(v, world, dev)
 
     name = args.workload
     if args.experts:
@@ -443,7 +459,7 @@ def run_ours(args):
         unit = "TFLOP/s"
         units_note = "2 * (T*k + S*T) * 2I * d"
     tokens = spec.T * world
-    value = tokens / (ms_step * 1e-3)
+    value = replica_throughput(spec.T, world, ms_total, K)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,

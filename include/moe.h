@@ -163,7 +163,8 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *top
 
 /* Grouped SwiGLU expert FFN over ragged groups (one expert per group):
  *   y[r] = (silu(a[r] W1_g^T) * (a[r] W3_g^T)) W2_g^T  for rows r of group g.
- *   n_groups        G (<= 1024); group g uses weights w13[g], w2[g]
+ *   n_groups        G (<= E + n_shared of cfg, which sizes the workspace); group g
+ *                   uses weights w13[g], w2[g]
  *   group_offsets   [G+1] int32 DEVICE array of row offsets into a / y
  *                   (non-decreasing; read on the device, never copied to the host).
  *                   Offsets that decrease or pass n_rows set the device status
@@ -210,6 +211,14 @@ MOE_API moe_status moe_layer_forward_staged(const moe_config *cfg, const moe_wei
                                             int32_t *topk_idx_out, float *topk_w_out, void *ws,
                                             size_t ws_bytes, cudaStream_t stream,
                                             cudaEvent_t *stage_events);
+
+/* Self-test of the device-side failure path (no counterpart on the pages): a
+ * tiny kernel waits on a barrier that nothing completes, gives up after
+ * `budget_cycles` SM clock cycles (1 .. 2^33), writes MOE_ERR_TIMEOUT into the
+ * status word of workspace `ws` and returns -- the bounded-wait path every
+ * tcgen05 kernel of the library takes instead of hanging.  Asynchronous; read
+ * the result with moe_read_device_status. */
+MOE_API moe_status moe_selftest_bounded_wait(void *ws, long long budget_cycles, cudaStream_t stream);
 
 /* Synchronises `stream`, then reads the device status word of workspace `ws`
  * into *out (MOE_OK when no device fault was recorded).  Does not clear it. */

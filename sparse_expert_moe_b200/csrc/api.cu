@@ -18,12 +18,14 @@ constexpr size_t kHeaderBytes = 256;
 constexpr int kHdrStatus = 0;
 constexpr int kHdrPermuteDone = 1;
 constexpr int kHdrNChunks = 2;
+constexpr int kHdrNGroups = 3;
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 // Byte offsets of every workspace region for one configuration.
 struct Layout {
-  size_t logits, topk_idx, topk_w, offsets, chunk_counts, perm_token, inv_perm, x_perm, chunks, h,
+  size_t logits, topk_idx, topk_w, offsets, chunk_counts, perm_token, inv_perm, x_perm, chunks,
+      grp_cp, h,
       y_rows, x_bf16, wr_bf16, w13_bf16, w2_bf16, a_bf16, x_sf, x_perm_sf, h_sf, a_sf, wsf13, wsf2,
       total;
   int64_t R, rows_all, n_chunk_max;
@@ -50,6 +52,7 @@ struct Layout {
     inv_perm = take(sizeof(int32_t) * R);
     x_perm = take(2 * R * d);
     chunks = take(sizeof(Chunk) * n_chunk_max);
+    grp_cp = take(sizeof(int32_t) * 2 * (E + S + 1));
     h = take(2 * rows_all * I);
     y_rows = take(2 * rows_all * d);
     x_bf16 = take(f32 || fp8 ? 2 * T * d : 0);
@@ -97,6 +100,13 @@ moe_status check_config(const moe_config* c) {
 }
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// bf16 chunk rows (= token-tile width of the expert GEMMs) for groups of at most
+// `max_group` rows: 32 for decode-sized batches, else 256 (FFN2 tiles of 256 tokens,
+// FFN1 tiles of half a chunk).
+int bf16_chunk_rows(int64_t max_group) {
+  return max_group <= kChunkRows ? kChunkRowsNarrow : kChunkRowsWide;
+}
 
 // ---------------------------------------------------------------- TMA maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -155,6 +165,19 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 
 namespace {
 
+// Token-operand maps with boxes of 128, 64, 32 and 16 rows.
+bool make_tok_maps(CUtensorMap (&m)[4], const void* base, uint64_t rows, uint64_t cols, bool u8) {
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t box = 128u >> i;
+    if (!(u8 ? make_tmap_u8(&m[i], base, rows, cols, box) : make_tmap_bf16(&m[i], base, rows, cols, box)))
+      return false;
+  }
+  return true;
+}
+void copy_maps(CUtensorMap (&dst)[4], const CUtensorMap (&src)[4]) {
+  for (int i = 0; i < 4; ++i) dst[i] = src[i];
+}
+
 // The FP8 block-scaled expert GEMMs over a chunk list already planned into the
 // workspace.  seg 0: routed rows a0 (token scales a0_sf [d/128][a0_rows]) with
 // weights w13_0 / w2_0 and their UE8M0 block scales wsf13_0 / wsf2_0 (G0 groups);
@@ -172,18 +195,20 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
   GemmLaunch g{};
   g.chunks = at<Chunk>(ws, L.chunks);
   g.n_chunks = at<int32_t>(ws, kHdrNChunks * sizeof(int));
+  g.grp_cp = at<int32_t>(ws, L.grp_cp);
+  g.n_grp = at<int32_t>(ws, kHdrNGroups * sizeof(int));
   g.status = status_word(ws);
   g.num_sms = num_sms();
 
   g.mode = kFFN1F8;
-  if (!make_tmap_u8(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) || !make_tmap_u8(&g.tmap[0], a0, a0_rows, d, 16))
+  if (!make_tmap_u8(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) || !make_tok_maps(g.tmap[0], a0, a0_rows, d, true))
     return MOE_ERR_CUDA;
   g.wsf[0] = wsf13_0;
   g.tsf[0] = a0_sf;
   g.tsf_ld[0] = static_cast<int>(a0_rows);
   g.tsf_rows[0] = static_cast<int>(a0_rows);
   if (S > 0) {
-    if (!make_tmap_u8(&g.wmap[1], w13_1, S * 2 * I, d, 128) || !make_tmap_u8(&g.tmap[1], a1, a1_rows, d, 16))
+    if (!make_tmap_u8(&g.wmap[1], w13_1, S * 2 * I, d, 128) || !make_tok_maps(g.tmap[1], a1, a1_rows, d, true))
       return MOE_ERR_CUDA;
     g.wsf[1] = wsf13_1;
     g.tsf[1] = a1_sf;
@@ -191,7 +216,7 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
     g.tsf_rows[1] = static_cast<int>(a1_rows);
   } else {
     g.wmap[1] = g.wmap[0];
-    g.tmap[1] = g.tmap[0];
+    copy_maps(g.tmap[1], g.tmap[0]);
     g.wsf[1] = g.wsf[0];
     g.tsf[1] = g.tsf[0];
     g.tsf_ld[1] = g.tsf_ld[0];
@@ -212,7 +237,7 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
   g.mode = kFFN2F8;
-  if (!make_tmap_u8(&g.wmap[0], w2_0, G0 * d, I, 128) || !make_tmap_u8(&g.tmap[0], h, rows_all, I, 16))
+  if (!make_tmap_u8(&g.wmap[0], w2_0, G0 * d, I, 128) || !make_tok_maps(g.tmap[0], h, rows_all, I, true))
     return MOE_ERR_CUDA;
   g.wsf[0] = wsf2_0;
   if (S > 0) {
@@ -222,7 +247,7 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
     g.wmap[1] = g.wmap[0];
     g.wsf[1] = g.wsf[0];
   }
-  g.tmap[1] = g.tmap[0];
+  copy_maps(g.tmap[1], g.tmap[0]);
   for (int i = 0; i < 2; ++i) {
     g.tsf[i] = h_sf;
     g.tsf_ld[i] = static_cast<int>(rows_all);
@@ -249,26 +274,33 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
 moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a0, int64_t a0_rows,
                    const void* w13_0, const void* w2_0, int64_t G0, const void* a1, int64_t a1_rows,
                    const void* w13_1, const void* w2_1, int64_t S, int64_t rows_all, void* y,
-                   cudaStream_t s, cudaEvent_t* ev = nullptr) {
+                   int chunk_rows, cudaStream_t s, cudaEvent_t* ev = nullptr) {
   const int64_t d = c.d_model, I = c.d_ff;
   void* h = at<void>(ws, L.h);
   GemmLaunch g{};
   g.chunks = at<Chunk>(ws, L.chunks);
   g.n_chunks = at<int32_t>(ws, kHdrNChunks * sizeof(int));
+  g.grp_cp = at<int32_t>(ws, L.grp_cp);
+  g.n_grp = at<int32_t>(ws, kHdrNGroups * sizeof(int));
   g.status = status_word(ws);
   g.num_sms = num_sms();
 
+  // FFN1 keeps 128-token tiles (two accumulator buffers overlap its SwiGLU epilogue with
+  // the next tile's MMAs); on 256-row chunks each tile takes half a chunk.  FFN2 runs
+  // 256-token tiles on them.
   g.mode = kFFN1;
+  g.tile_tokens = chunk_rows == kChunkRowsWide ? kChunkRows : chunk_rows;
+  g.halves = chunk_rows == kChunkRowsWide;
   if (!make_tmap_bf16(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) ||
-      !make_tmap_bf16(&g.tmap[0], a0, a0_rows, d, 16))
+      !make_tok_maps(g.tmap[0], a0, a0_rows, d, false))
     return MOE_ERR_CUDA;
   if (S > 0) {
     if (!make_tmap_bf16(&g.wmap[1], w13_1, S * 2 * I, d, 128) ||
-        !make_tmap_bf16(&g.tmap[1], a1, a1_rows, d, 16))
+        !make_tok_maps(g.tmap[1], a1, a1_rows, d, false))
       return MOE_ERR_CUDA;
   } else {
     g.wmap[1] = g.wmap[0];
-    g.tmap[1] = g.tmap[0];
+    copy_maps(g.tmap[1], g.tmap[0]);
   }
   g.n_mblk = static_cast<int>(I / 128);
   g.k_blocks = static_cast<int>(d / 64);
@@ -282,15 +314,17 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
   g.mode = kFFN2;
+  g.tile_tokens = chunk_rows;
+  g.halves = false;
   if (!make_tmap_bf16(&g.wmap[0], w2_0, G0 * d, I, 128) ||
-      !make_tmap_bf16(&g.tmap[0], h, rows_all, I, 16))
+      !make_tok_maps(g.tmap[0], h, rows_all, I, false))
     return MOE_ERR_CUDA;
   if (S > 0) {
     if (!make_tmap_bf16(&g.wmap[1], w2_1, S * d, I, 128)) return MOE_ERR_CUDA;
   } else {
     g.wmap[1] = g.wmap[0];
   }
-  g.tmap[1] = g.tmap[0];
+  copy_maps(g.tmap[1], g.tmap[0]);
   g.n_mblk = static_cast<int>(d / 128);
   g.k_blocks = static_cast<int>(I / 64);
   g.w_rows_per_group = static_cast<int>(d);
@@ -367,6 +401,8 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
   if (!aligned16(a) || !aligned16(w13) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   const Layout L(*cfg);
   if (n_rows > L.rows_all) return MOE_ERR_UNSUPPORTED;
+  // the workspace's chunk list and group tables are sized for E + n_shared groups
+  if (n_groups > cfg->E + cfg->n_shared) return MOE_ERR_UNSUPPORTED;
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   if (n_rows == 0) return MOE_OK;
   const int64_t d = cfg->d_model, I = cfg->d_ff;
@@ -374,7 +410,6 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
   const void* w13_b = w13;
   const void* w2_b = w2;
   if (cfg->act == MOE_F32) {
-    if (n_groups > cfg->E + cfg->n_shared) return MOE_ERR_UNSUPPORTED;
     st = cuda_status(launch_f32_to_bf16(static_cast<const float*>(a), at<void>(ws, L.a_bf16),
                                         static_cast<size_t>(n_rows) * d, stream));
     if (st == MOE_OK)
@@ -390,7 +425,6 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
   }
   if (cfg->act == MOE_E4M3) {
     if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
-    if (n_groups > cfg->E + cfg->n_shared) return MOE_ERR_UNSUPPORTED;
     uint32_t* a_sf = at<uint32_t>(ws, L.a_sf);
     uint4* wsf13 = at<uint4>(ws, L.wsf13);
     uint4* wsf2 = at<uint4>(ws, L.wsf2);
@@ -405,17 +439,20 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
     if (st == MOE_OK)
       st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRowsFP8,
                                    at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                               at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
                                    status_word(ws), stream));
     if (st != MOE_OK) return st;
     return run_ffn_fp8(*cfg, L, ws, a, a_sf, n_rows, w13, w2, wsf13, wsf2, n_groups, nullptr,
                        nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0, n_rows, y, stream);
   }
-  st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRows,
+  const int chunk_rows = bf16_chunk_rows(n_rows);
+  st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, chunk_rows,
                                at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                               at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
                                status_word(ws), stream));
   if (st != MOE_OK) return st;
   return run_ffn(*cfg, L, ws, a_b, n_rows, w13_b, w2_b, n_groups, nullptr, 0, nullptr, nullptr, 0,
-                 n_rows, y, stream);
+                 n_rows, y, chunk_rows, stream);
 }
 
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* inv_perm,
@@ -515,10 +552,10 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   {
     GemmLaunch g{};
     g.mode = kRouter;
-    if (!make_tmap_bf16(&g.wmap[0], wr_b, E, d, 128) || !make_tmap_bf16(&g.tmap[0], x_router, T, d, 16))
+    if (!make_tmap_bf16(&g.wmap[0], wr_b, E, d, 128) || !make_tok_maps(g.tmap[0], x_router, T, d, false))
       return MOE_ERR_CUDA;
     g.wmap[1] = g.wmap[0];
-    g.tmap[1] = g.tmap[0];
+    copy_maps(g.tmap[1], g.tmap[0]);
     g.router_T = static_cast<int>(T);
     g.n_mblk = static_cast<int>((E + 127) / 128);
     g.k_blocks = static_cast<int>(d / 64);
@@ -559,10 +596,13 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if (st != MOE_OK) return st;
   if ((st = mark(3)) != MOE_OK) return st;
 
-  // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs
+  // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs.  Groups hold at
+  // most T rows, which picks the bf16 token-tile width.
+  const int chunk_rows = fp8 ? kChunkRowsFP8 : bf16_chunk_rows(T);
   st = cuda_status(launch_plan(offsets, c.E, static_cast<int>(R), c.n_shared, c.T,
-                               static_cast<int>(R), fp8 ? kChunkRowsFP8 : kChunkRows,
+                               static_cast<int>(R), chunk_rows,
                                at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                               at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
                                status, s));
   if (st != MOE_OK) return st;
   if ((st = mark(4)) != MOE_OK) return st;
@@ -575,7 +615,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
                      ev ? ev + 5 : nullptr);
   } else {
     st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows,
-                 s, ev ? ev + 5 : nullptr);
+                 chunk_rows, s, ev ? ev + 5 : nullptr);
   }
   if (st != MOE_OK) return st;
 

@@ -42,16 +42,20 @@ namespace {
 
 constexpr int kBM = 128;                  // weight rows per tile (UMMA M)
 constexpr int kRowBytes = 128;            // K bytes per stage and row: one 128-byte swizzle row
-constexpr int kTokBox = 16;               // token rows per TMA box
 constexpr uint32_t kABytes = kBM * kRowBytes;
-constexpr uint32_t kTokBoxBytes = kTokBox * kRowBytes;
 constexpr uint32_t kSFAtomBytes = 512;    // 128 rows x 4 UE8M0 bytes (tcgen05.cp 32x128b source)
+
+constexpr int kTokBoxes = 4;              // token boxes of 128, 64, 32, 16 rows
 
 struct DevParams {
   CUtensorMap wmap[2];
-  CUtensorMap tmap[2];
+  CUtensorMap tmap[2][kTokBoxes];
   const Chunk* chunks;
   const int32_t* n_chunks;
+  const int32_t* grp_cp;      // chunk prefix of the planned groups (largest first) [n_grp + 1],
+                              // then their half-chunk prefix [n_grp + 1]
+  const int32_t* n_grp;
+  int halves;                 // chunks hold 2 x kNT rows: each tile takes one non-empty half
   int router_T;
   int n_mblk;
   int k_blocks;
@@ -74,52 +78,116 @@ struct DevParams {
   int ld_out_sf;
 };
 
-template <int MODE>
+// NTW: token-tile width of the bf16 expert GEMMs.  128 by default; 32 for decode-sized
+// batches (small shared-memory token tiles leave room for a deeper weight ring: 5 / 9
+// stages); 256 for large groups (twice the reuse of every weight byte loaded into
+// shared memory; a 256-wide FFN1 would hold its gate and up accumulators in all 512
+// TMEM columns -- one buffer -- so FFN1 instead takes half a 256-row chunk per tile).
+template <int MODE, int NTW = kChunkRows>
 struct Cfg {
   static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8;
   static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8;   // gate + up accumulators
+  static_assert(NTW == kChunkRows || !(kFP8 || MODE == kRouter), "tile width: bf16 expert GEMMs");
   static constexpr int kATiles = kGLU ? 2 : 1;
-  static constexpr int kNT = kFP8 ? kChunkRowsFP8 : kChunkRows;     // max tokens per tile
+  static constexpr int kNT = kFP8 ? kChunkRowsFP8 : NTW;
+  static constexpr int kAccBufs = (kGLU && kNT > 128) ? 1 : 2;
   static constexpr uint32_t kBBytes = kNT * kRowBytes;
   static constexpr uint32_t kSFBytes = kFP8 ? (kATiles + 1) * kSFAtomBytes : 0;
   static constexpr uint32_t kStageBytes =
       ((kATiles * kABytes + kBBytes + kSFBytes + 1023) / 1024) * 1024;
-  static constexpr int kStages = kGLU ? 4 : 6;
+  static constexpr int kStagesFit = static_cast<int>((192u * 1024u) / kStageBytes);
+  static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
   static constexpr uint32_t kAccCols = kGLU ? 2 * kNT : kNT;        // per accumulator buffer
   static constexpr uint32_t kSFColsPerStage = 16;                     // <= 3 atoms x 4 columns
   static constexpr uint32_t kSFCols = kFP8 ? kStages * kSFColsPerStage : 0;
-  static constexpr uint32_t kColsUsed = 2 * kAccCols + kSFCols;
-  static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256 : 512;
+  static constexpr uint32_t kColsUsed = kAccBufs * kAccCols + kSFCols;
+  static constexpr uint32_t kTmemCols =
+      kColsUsed <= 64 ? 64 : (kColsUsed <= 128 ? 128 : (kColsUsed <= 256 ? 256 : 512));
   static constexpr int kThreads = kFP8 ? 224 : 192;                 // + one scale-factor warp
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
+  static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;      // per epilogue warp: 16 x 32 x 4 B
+  static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;   // group (half-)chunk prefixes
+  static constexpr uint32_t kRedBytes = kFP8 ? 2 * 4 * 128 * 4 : 0;  // FP8 amax exchange
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + kStagingBytes +
+                                         kGrpBytes + 16 + kRedBytes + 1024 /*align*/;
   static_assert(kColsUsed <= 512, "TMEM budget");
 };
 
 template <int MODE>
 __device__ __forceinline__ Chunk get_chunk(const DevParams& p, int ci) {
   if (p.chunks) return p.chunks[ci];
-  Chunk c;
+  Chunk c;                                   // router: fixed chunks of kChunkRows tokens
   c.seg = 0;
   c.group = 0;
-  c.b_row = ci * Cfg<MODE>::kNT;
+  c.b_row = ci * kChunkRows;
   c.o_row = c.b_row;
-  c.nrows = min(Cfg<MODE>::kNT, p.router_T - c.b_row);
+  c.nrows = min(kChunkRows, p.router_T - c.b_row);
   return c;
 }
 
-// Tile t -> (chunk, weight block, K split).  Splits are fastest, then weight blocks.
+// Tile t -> (chunk, weight block, K split).
+// Router (no chunk list): splits fastest, then weight blocks, then token chunks.
+// Grouped GEMMs: tiles are laid out group by group (largest group first); inside a
+// group of c chunks and n_mblk weight blocks, blocks of G weight blocks (G = 4 when
+// it divides n_mblk) sweep all c chunks before the next G: CTAs running at the same
+// time share a few weight blocks and many token chunks, both resident in L2, so an
+// expert's weights and tokens come from HBM about once.
+
 struct TileCoord {
-  int chunk, mb, split, kb0, kb1;
+  int chunk, mb, split, kb0, kb1, half;
 };
-__device__ __forceinline__ TileCoord tile_coord(const DevParams& p, int t) {
+__device__ __forceinline__ TileCoord tile_coord(const DevParams& p, int t, const int32_t* cp,
+                                                int n_grp) {
+  // cp: chunk prefix [n_grp + 1] followed by the half-chunk prefix [n_grp + 1]
   TileCoord tc;
-  tc.split = t % p.k_splits;
-  const int r = t / p.k_splits;
-  tc.chunk = r / p.n_mblk;
-  tc.mb = r % p.n_mblk;
-  tc.kb0 = tc.split * p.k_per_split;
-  tc.kb1 = min(p.k_blocks, tc.kb0 + p.k_per_split);
+  tc.half = 0;
+  if (!p.chunks) {
+    tc.split = t % p.k_splits;
+    const int r = t / p.k_splits;
+    tc.chunk = r / p.n_mblk;
+    tc.mb = r % p.n_mblk;
+    tc.kb0 = tc.split * p.k_per_split;
+    tc.kb1 = min(p.k_blocks, tc.kb0 + p.k_per_split);
+    return tc;
+  }
+  const int n = p.n_mblk;
+  const int32_t* up = p.halves ? cp + n_grp + 1 : cp;   // units: chunks or half chunks
+  int lo = 0, hi = n_grp;                                // up[lo] * n <= t < up[hi] * n
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (up[mid] * n <= t) lo = mid; else hi = mid;
+  }
+  const int cg = up[lo + 1] - up[lo];
+  const int local = t - up[lo] * n;
+  const int G = (n % 4 == 0) ? 4 : ((n % 2 == 0) ? 2 : 1);
+  const int blk = cg * G;
+  const int mbb = local / blk, rem = local - mbb * blk;
+  const int unit = rem / G;                              // chunk (or half chunk) in the group
+  tc.mb = mbb * G + rem % G;
+  if (p.halves) {
+    tc.chunk = cp[lo] + (unit >> 1);
+    tc.half = unit & 1;
+  } else {
+    tc.chunk = cp[lo] + unit;
+  }
+  tc.split = 0;
+  tc.kb0 = 0;
+  tc.kb1 = p.k_blocks;
   return tc;
+}
+
+// The rows a tile covers: its chunk, or one half of it when chunks are twice the
+// tile width (nrows <= 0: nothing to do -- every role skips the tile alike).
+template <int MODE>
+__device__ __forceinline__ Chunk tile_rows(const DevParams& p, const TileCoord& tc) {
+  Chunk c = get_chunk<MODE>(p, tc.chunk);
+  if (p.halves) {
+    const int off = tc.half * Cfg<MODE>::kNT;
+    c.b_row += off;
+    c.o_row += off;
+    c.nrows -= off;
+    if (c.nrows > Cfg<MODE>::kNT) c.nrows = Cfg<MODE>::kNT;
+  }
+  return c;
 }
 
 // Smallest e with amax <= 448 * 2^e (amax as fp32 bits, non-negative), clamped to the
@@ -133,10 +201,33 @@ __device__ __forceinline__ int e4m3_scale_exponent(uint32_t amax_bits) {
   return max(-127, min(127, e));
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
+// Writes a warp's 16 (rows) x 32 (columns) output block: each lane holds one column's
+// 16 values; they pass through the warp's shared-memory staging area so that global
+// memory sees 16-byte vector stores (each row's 32 elements are contiguous), rows at
+// or past `nvalid` skipped.  `g` points at element (row 0, column 0) of the block;
+// `ld` is the row pitch in elements (the pitch and `g` must be 16-byte aligned).
+template <typename T>
+__device__ __forceinline__ void store_block_16x32(T* g, int ld, int nvalid, const T (&v)[16],
+                                                  T* stage, int lane) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) stage[i * 32 + lane] = v[i];
+  __syncwarp();
+  constexpr int kVecPerRow = 32 * static_cast<int>(sizeof(T)) / 16;
+  constexpr int kElemPerVec = 16 / static_cast<int>(sizeof(T));
+#pragma unroll
+  for (int q = lane; q < 16 * kVecPerRow; q += 32) {
+    const int row = q / kVecPerRow, cv = q % kVecPerRow;
+    if (row < nvalid)
+      *reinterpret_cast<uint4*>(g + static_cast<size_t>(row) * ld + cv * kElemPerVec) =
+          *reinterpret_cast<const uint4*>(stage + row * 32 + cv * kElemPerVec);
+  }
+  __syncwarp();
+}
+
+template <int MODE, int NTW>
+__global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ DevParams p) {
-  using C = Cfg<MODE>;
+  using C = Cfg<MODE, NTW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -148,7 +239,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
   uint64_t* red_bar = tempty_bar + 2;                            // [2] FP8 amax exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* red = reinterpret_cast<uint32_t*>(tmem_slot + 4);   // [2][4][16] FP8 amax exchange
+  uint8_t* staging = smem + C::kStages * C::kStageBytes + 1024;  // [4 warps][16 x 32 x 4 B]
+  int32_t* grp_cp = reinterpret_cast<int32_t*>(staging + C::kStagingBytes);
+  // FP8: [2 buffers][4 warps][128 tokens] per-warp amax of the tile's h values
+  uint32_t* red = reinterpret_cast<uint32_t*>(staging + C::kStagingBytes + C::kGrpBytes + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -166,7 +260,12 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.wmap[0]);
-    tma_prefetch_desc(&p.tmap[0]);
+    tma_prefetch_desc(&p.tmap[0][0]);
+  }
+  int n_grp = 0;
+  if (p.chunks) {
+    n_grp = *p.n_grp;
+    for (int i = threadIdx.x; i < 2 * (n_grp + 1); i += blockDim.x) grp_cp[i] = p.grp_cp[i];
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -177,8 +276,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_chunks = p.chunks ? *p.n_chunks : (p.router_T + C::kNT - 1) / C::kNT;
-  const int n_tiles = n_chunks * p.n_mblk * p.k_splits;
+  const int n_chunks = p.chunks ? *p.n_chunks : (p.router_T + kChunkRows - 1) / kChunkRows;
+  const int n_units = !p.chunks ? n_chunks : (p.halves ? grp_cp[2 * n_grp + 1] : n_chunks);
+  const int n_tiles = n_units * p.n_mblk * (p.chunks ? 1 : p.k_splits);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -186,16 +286,16 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const TileCoord tc = tile_coord(p, t);
-        const Chunk c = get_chunk<MODE>(p, tc.chunk);
+        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+        const Chunk c = tile_rows<MODE>(p, tc);
+        if (c.nrows <= 0) continue;
         const int mb = tc.mb;
         const int a_row = c.group * p.w_rows_per_group + mb * kBM;
-        const int nbox = (c.nrows + kTokBox - 1) / kTokBox;
+        const int n_pad = (c.nrows + 15) & ~15;
         // the second GEMM reads the h rows the first one wrote (output numbering)
         const int tok_row = (MODE == kFFN2 || MODE == kFFN2F8) ? c.o_row : c.b_row;
-        const uint32_t bytes = C::kATiles * kABytes + nbox * kTokBoxBytes;
+        const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;
         const CUtensorMap* wm = &p.wmap[c.seg];
-        const CUtensorMap* tm = &p.tmap[c.seg];
         for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -207,8 +307,14 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           tma_load_2d(st, wm, &full_bar[stage], kx, a_row);
           if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[stage], kx, a_row + p.up_offset);
           uint8_t* bt = st + C::kATiles * kABytes;
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(bt + i * kTokBoxBytes, tm, &full_bar[stage], kx, tok_row + i * kTokBox);
+          // token rows as boxes of 128 / 64 / 32 / 16 rows covering n_pad
+          for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
+            const int rows = 128 >> bi;
+            while (n_pad - off >= rows) {
+              tma_load_2d(bt + off * kRowBytes, &p.tmap[c.seg][bi], &full_bar[stage], kx, tok_row + off);
+              off += rows;
+            }
+          }
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
@@ -223,13 +329,14 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int it = 0;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const TileCoord tc = tile_coord(p, t);
-        const Chunk c = get_chunk<MODE>(p, tc.chunk);
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+        const Chunk c = tile_rows<MODE>(p, tc);
+        if (c.nrows <= 0) continue;
         const int n_pad = (c.nrows + 15) & ~15;
         const uint32_t idesc = C::kFP8 ? idesc_e4m3_bs(kBM, n_pad) : idesc_bf16_f32(kBM, n_pad);
-        const uint32_t acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const uint32_t acc = it % C::kAccBufs;
+        const uint32_t acc_phase = (it / C::kAccBufs) & 1;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
@@ -246,7 +353,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
             // scale factors of this stage: smem (written by the scale warp) -> TMEM
             fence_proxy_async_smem();
             const uint32_t sf_smem = bt + C::kBBytes;
-            const uint32_t sfa = tmem_base + 2 * C::kAccCols + stage * C::kSFColsPerStage;
+            const uint32_t sfa = tmem_base + C::kAccBufs * C::kAccCols + stage * C::kSFColsPerStage;
             const uint32_t sfb = sfa + C::kATiles * 4;
             tmem_cp_32x128b_warpx4(sfa, smem_desc_noswizzle(sf_smem));
             if (C::kGLU) tmem_cp_32x128b_warpx4(sfa + 4, smem_desc_noswizzle(sf_smem + kSFAtomBytes));
@@ -276,6 +383,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           }
         }
         if (ok) umma_commit(&tfull_bar[acc]);
+        ++it;
       }
     }
     __syncwarp();
@@ -286,73 +394,85 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     int it = 0;
     uint32_t rbuf = 0, rpar = 0;              // FP8 amax exchange: buffer and per-buffer parity bits
     bool epi_ok = true;
-    for (int t = blockIdx.x; t < n_tiles && epi_ok; t += gridDim.x, ++it) {
-      const TileCoord tc = tile_coord(p, t);
-      const Chunk c = get_chunk<MODE>(p, tc.chunk);
+    for (int t = blockIdx.x; t < n_tiles && epi_ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+      const Chunk c = tile_rows<MODE>(p, tc);
+      if (c.nrows <= 0) continue;
       const int mb = tc.mb;
-      const uint32_t acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const uint32_t acc = it % C::kAccBufs;
+      const uint32_t acc_phase = (it / C::kAccBufs) & 1;
       bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + acc * C::kAccCols;
       const int m = mb * kBM + m_local;       // output column
-      for (int n0 = 0; n0 < c.nrows; n0 += 16) {
+      if (MODE == kFFN1F8) {
+        // SwiGLU, then requantise h to e4m3 with one power-of-two scale per token per 128
+        // h columns (this tile's columns).  Pass 1: per token, the maximum |h| of each
+        // warp's 32 columns (redux.sync) into shared memory; one exchange between the
+        // four epilogue warps (mbarrier, bounded wait); pass 2: reload the accumulators,
+        // recompute h, scale, round to e4m3 and store with the scales.
+        uint32_t* redt = red + rbuf * (4 * 128);
+        for (int n0 = 0; n0 < c.nrows; n0 += 16) {
+          float g[16], u[16];
+          tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float hv = g[i] / (1.0f + __expf(-g[i])) * u[i];
+            const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv)));
+            if (lane == 0) redt[sub * 128 + n0 + i] = wmax;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_bar[rbuf]);
+        const bool rok = mbar_wait(&red_bar[rbuf], (rpar >> rbuf) & 1u, abort_flag, p.status);
+        rpar ^= 1u << rbuf;
+        if (!__all_sync(0xffffffffu, rok)) {
+          epi_ok = false;
+        } else {
+          for (int n0 = 0; n0 < c.nrows; n0 += 16) {
+            float g[16], u[16];
+            tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
+            uint8_t q[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float hv = g[i] / (1.0f + __expf(-g[i])) * u[i];
+              const int n = n0 + i;
+              const uint32_t amax = max(max(redt[n], redt[128 + n]), max(redt[256 + n], redt[384 + n]));
+              const int e = e4m3_scale_exponent(amax);
+              q[i] = __nv_cvt_float_to_fp8(scalbnf(hv, -e), __NV_SATFINITE, __NV_E4M3);
+              if (m_local == 0 && n < c.nrows)
+                p.out_sf[static_cast<size_t>(mb) * p.ld_out_sf + c.o_row + n] =
+                    0x01010101u * static_cast<uint32_t>(e + 127);
+            }
+            store_block_16x32(static_cast<uint8_t*>(p.out) +
+                                  static_cast<size_t>(c.o_row + n0) * p.ld_out + (m - lane),
+                              p.ld_out, c.nrows - n0, q, staging + sub * 2048, lane);
+          }
+        }
+        rbuf ^= 1u;
+      }
+      for (int n0 = 0; n0 < c.nrows && MODE != kFFN1F8; n0 += 16) {
         if (MODE == kFFN1) {
           float g[16], u[16];
           tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
-          __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out);
+          __nv_bfloat16 hv[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (n0 + i < c.nrows) {
-              const float s = g[i] / (1.0f + __expf(-g[i]));
-              h[static_cast<size_t>(c.o_row + n0 + i) * p.ld_out + m] = __float2bfloat16_rn(s * u[i]);
-            }
-          }
-        } else if (MODE == kFFN1F8) {
-          // SwiGLU, then requantise h to e4m3 with one power-of-two scale per token per
-          // 128 h columns (this tile's columns): amax across the tile's 128 threads, the
-          // four warps' partial maxima exchanged through shared memory (double-buffered,
-          // one mbarrier per buffer, bounded waits)
-          float g[16], u[16], hv[16];
-          tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            hv[i] = g[i] / (1.0f + __expf(-g[i])) * u[i];
-            const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[i])));
-            if (lane == 0) red[(rbuf * 4 + sub) * 16 + i] = wmax;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&red_bar[rbuf]);
-          const bool rok = mbar_wait(&red_bar[rbuf], (rpar >> rbuf) & 1u, abort_flag, p.status);
-          rpar ^= 1u << rbuf;
-          if (!__all_sync(0xffffffffu, rok)) {
-            epi_ok = false;
-            break;
-          }
-          uint8_t* h = static_cast<uint8_t*>(p.out);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint32_t* r = red + rbuf * 64 + i;
-            const uint32_t amax = max(max(r[0], r[16]), max(r[32], r[48]));
-            const int e = e4m3_scale_exponent(amax);
-            if (n0 + i < c.nrows) {
-              const __nv_fp8_storage_t q = __nv_cvt_float_to_fp8(scalbnf(hv[i], -e), __NV_SATFINITE, __NV_E4M3);
-              h[static_cast<size_t>(c.o_row + n0 + i) * p.ld_out + m] = q;
-              if (m_local == 0)
-                p.out_sf[static_cast<size_t>(mb) * p.ld_out_sf + c.o_row + n0 + i] =
-                    0x01010101u * static_cast<uint32_t>(e + 127);
-            }
-          }
-          rbuf ^= 1u;
+          for (int i = 0; i < 16; ++i) hv[i] = __float2bfloat16_rn(g[i] / (1.0f + __expf(-g[i])) * u[i]);
+          store_block_16x32(static_cast<__nv_bfloat16*>(p.out) +
+                                static_cast<size_t>(c.o_row + n0) * p.ld_out + (m - lane),
+                            p.ld_out, c.nrows - n0, hv,
+                            reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
         } else if (MODE == kFFN2 || MODE == kFFN2F8) {
           float v[16];
           tmem_ld16(tb + n0, v);
-          __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.out);
+          __nv_bfloat16 yv[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (n0 + i < c.nrows)
-              y[static_cast<size_t>(c.o_row + n0 + i) * p.ld_out + m] = __float2bfloat16_rn(v[i]);
+          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v[i]);
+          store_block_16x32(static_cast<__nv_bfloat16*>(p.out) +
+                                static_cast<size_t>(c.o_row + n0) * p.ld_out + (m - lane),
+                            p.ld_out, c.nrows - n0, yv,
+                            reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
         } else {
           float v[16];
           tmem_ld16(tb + n0, v);
@@ -366,6 +486,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
+      ++it;
     }
   } else if (C::kFP8) {
     // ------------------------------------------------------------ scale-factor warp (FP8)
@@ -377,8 +498,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     bool ok = true;
     const int up_rb = p.up_offset / kBM;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-      const TileCoord tc = tile_coord(p, t);
-      const Chunk c = get_chunk<MODE>(p, tc.chunk);
+      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+      const Chunk c = tile_rows<MODE>(p, tc);
+      if (c.nrows <= 0) continue;
       const int mb = tc.mb;
       const int n_pad = (c.nrows + 15) & ~15;
       const int tok_row = MODE == kFFN2F8 ? c.o_row : c.b_row;
@@ -421,6 +543,33 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- planner
+// Exclusive block-wide scan (1024 threads, <= 2048 entries) of ceil(sz[order[r]] / rows)
+// over ranks r, into base[0..NG].
+__device__ void block_scan_counts(const int32_t* sz, const int32_t* order, int NG, int rows,
+                                  int32_t* base, int32_t* warp_sum) {
+  const int tid = threadIdx.x;
+  int c0 = 0, c1 = 0;
+  const int r0 = 2 * tid, r1 = 2 * tid + 1;
+  if (r0 < NG) c0 = (sz[order[r0]] + rows - 1) / rows;
+  if (r1 < NG) c1 = (sz[order[r1]] + rows - 1) / rows;
+  const int local = c0 + c1;
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = local;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int wb = 0;
+  for (int w = 0; w < warp; ++w) wb += warp_sum[w];
+  const int excl = wb + incl - local;
+  if (r0 < NG) base[r0] = excl;
+  if (r1 < NG) base[r1] = excl + c0;
+  if (tid == blockDim.x - 1) base[NG] = excl + local;
+  __syncthreads();
+}
+
 // One CTA.  Validates the offsets, orders the groups by size (largest first,
 // ties by index: routed before shared), splits each into chunks of at most
 // `cr` rows (the GEMM's token tile) and writes the chunk list and its length.
@@ -428,11 +577,14 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
                                                     int n_rows, int n_shared, int T,
                                                     int shared_o_row, int cr,
                                                     Chunk* __restrict__ chunks,
-                                                    int32_t* __restrict__ n_chunks, int* status) {
+                                                    int32_t* __restrict__ n_chunks,
+                                                    int32_t* __restrict__ grp_cp,
+                                                    int32_t* __restrict__ n_grp, int* status) {
   __shared__ int32_t sz[kMaxGroups];
   __shared__ int32_t start[kMaxGroups];
   __shared__ int32_t order[kMaxGroups];
   __shared__ int32_t cbase[kMaxGroups + 1];
+  __shared__ int32_t hbase[kMaxGroups + 1];
   __shared__ int bad;
   __shared__ int32_t warp_sum[32];
   const int NG = G + n_shared;
@@ -458,6 +610,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     if (tid == 0) {
       record_status(status, kStatusDeviceIndex);
       *n_chunks = 0;
+      *n_grp = 0;
+      grp_cp[0] = 0;
+      grp_cp[1] = 0;
     }
     return;
   }
@@ -471,27 +626,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     order[rank] = g;
   }
   __syncthreads();
-  // exclusive scan of chunk counts in rank order; thread owns ranks 2*tid, 2*tid+1
-  int c0 = 0, c1 = 0;
-  const int r0 = 2 * tid, r1 = 2 * tid + 1;
-  if (r0 < NG) c0 = (sz[order[r0]] + cr - 1) / cr;
-  if (r1 < NG) c1 = (sz[order[r1]] + cr - 1) / cr;
-  const int local = c0 + c1;
-  const int lane = tid & 31, warp = tid >> 5;
-  int incl = local;
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) warp_sum[warp] = incl;
-  __syncthreads();
-  int wb = 0;
-  for (int w = 0; w < warp; ++w) wb += warp_sum[w];
-  const int excl = wb + incl - local;
-  if (r0 < NG) cbase[r0] = excl;
-  if (r1 < NG) cbase[r1] = excl + c0;
-  if (tid == blockDim.x - 1) cbase[NG] = excl + local;
-  __syncthreads();
+  // exclusive scans, in rank order, of the chunk counts (chunks of cr rows) and of the
+  // half-chunk counts (cr / 2 rows)
+  block_scan_counts(sz, order, NG, cr, cbase, warp_sum);
+  block_scan_counts(sz, order, NG, cr / 2, hbase, warp_sum);
   for (int r = tid; r < NG; r += blockDim.x) {
     const int g = order[r];
     const int s = sz[g];
@@ -508,30 +646,40 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
       chunks[base + c] = ch;
     }
   }
-  if (tid == 0) *n_chunks = cbase[NG];
+  for (int r = tid; r <= NG; r += blockDim.x) {
+    grp_cp[r] = cbase[r];
+    grp_cp[NG + 1 + r] = hbase[r];
+  }
+  if (tid == 0) {
+    *n_chunks = cbase[NG];
+    *n_grp = NG;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared, int T,
                         int shared_o_row, int chunk_rows, Chunk* chunks, int32_t* n_chunks,
-                        int* status, cudaStream_t s) {
+                        int32_t* grp_cp, int32_t* n_grp, int* status, cudaStream_t s) {
   plan_kernel<<<1, 1024, 0, s>>>(offsets, G, n_rows, n_shared, T, shared_o_row, chunk_rows, chunks,
-                                 n_chunks, status);
+                                 n_chunks, grp_cp, n_grp, status);
   return cudaGetLastError();
 }
 
-template <int MODE>
+template <int MODE, int NTW>
 static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
-  using C = Cfg<MODE>;
+  using C = Cfg<MODE, NTW>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
   DevParams p;
   p.wmap[0] = g.wmap[0];
   p.wmap[1] = g.wmap[1];
-  p.tmap[0] = g.tmap[0];
-  p.tmap[1] = g.tmap[1];
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < kTokBoxes; ++j) p.tmap[i][j] = g.tmap[i][j];
   p.chunks = g.chunks;
   p.n_chunks = g.n_chunks;
+  p.grp_cp = g.grp_cp;
+  p.n_grp = g.n_grp;
+  p.halves = g.halves ? 1 : 0;
   p.router_T = g.router_T;
   p.n_mblk = g.n_mblk;
   p.k_blocks = g.k_blocks;
@@ -553,27 +701,32 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   p.wsf_rb_per_group = g.wsf_rb_per_group;
   p.out_sf = g.out_sf;
   p.ld_out_sf = g.ld_out_sf;
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, NTW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::kSmemBytes));
   if (err != cudaSuccess) return err;
   int grid = g.num_sms;
   if (MODE == kRouter) {
-    const int tiles = ((g.router_T + C::kNT - 1) / C::kNT) * g.n_mblk * p.k_splits;
+    const int tiles = ((g.router_T + kChunkRows - 1) / kChunkRows) * g.n_mblk * p.k_splits;
     if (tiles < grid) grid = tiles;
     if (grid == 0) return cudaSuccess;
   }
-  grouped_gemm_kernel<MODE><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
+  grouped_gemm_kernel<MODE, NTW><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   switch (g.mode) {
-    case kRouter: return launch_mode<kRouter>(g, s);
-    case kFFN1: return launch_mode<kFFN1>(g, s);
-    case kFFN2: return launch_mode<kFFN2>(g, s);
-    case kFFN1F8: return launch_mode<kFFN1F8>(g, s);
-    case kFFN2F8: return launch_mode<kFFN2F8>(g, s);
+    case kRouter: return launch_mode<kRouter, kChunkRows>(g, s);
+    case kFFN1:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1, kChunkRowsNarrow>(g, s);
+      return launch_mode<kFFN1, kChunkRows>(g, s);
+    case kFFN2:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2, kChunkRowsNarrow>(g, s);
+      if (g.tile_tokens == kChunkRowsWide) return launch_mode<kFFN2, kChunkRowsWide>(g, s);
+      return launch_mode<kFFN2, kChunkRows>(g, s);
+    case kFFN1F8: return launch_mode<kFFN1F8, kChunkRows>(g, s);
+    case kFFN2F8: return launch_mode<kFFN2F8, kChunkRows>(g, s);
     default: return cudaErrorInvalidValue;
   }
 }

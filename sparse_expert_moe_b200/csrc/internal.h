@@ -26,10 +26,12 @@ struct Chunk {
 
 constexpr int kChunkRows = 128;     // tokens per GEMM tile, bf16 (UMMA N <= 128)
 constexpr int kChunkRowsFP8 = 112;  // tokens per GEMM tile, FP8 (TMEM also holds scale factors)
+constexpr int kChunkRowsWide = 256; // tokens per GEMM tile, bf16 wide tiles (groups > 128 rows)
+constexpr int kChunkRowsNarrow = 32; // tokens per GEMM tile, bf16 decode-sized batches
 constexpr int kMaxGroups = 1024 + 8;
 
 // Upper bound on the chunks of `rows` rows spread over `groups` groups.
-inline int64_t max_chunks(int64_t rows, int64_t groups, int chunk_rows = kChunkRowsFP8) {
+inline int64_t max_chunks(int64_t rows, int64_t groups, int chunk_rows = kChunkRowsNarrow) {
   return rows / chunk_rows + groups + 1;
 }
 
@@ -40,13 +42,14 @@ cudaError_t launch_route(const float* logits, int n_partials, long long partial_
                          const float* sel_bias, int T, int E, int k, int score, int32_t* topk_idx,
                          float* topk_w, cudaStream_t s);
 
-// K splits of the router GEMM for T tokens, E experts and d_model: enough CTAs to
-// cover the 148 SMs when the (token chunk, expert block) tiles alone cannot;
-// every split non-empty.  Host only.
+// K splits of the router GEMM for T tokens, E experts and d_model: about 48 CTAs
+// when the (token chunk, expert block) tiles alone are fewer -- enough to stream
+// Wr quickly, few enough that summing the partial logits stays cheap; every split
+// non-empty.  Host only.
 inline int router_splits(int64_t T, int64_t E, int64_t d) {
   const int64_t tiles = ((T + 127) / 128) * ((E + 127) / 128);
   const int64_t kb = d / 64;
-  int64_t s = tiles >= 148 ? 1 : 148 / tiles;
+  int64_t s = tiles >= 48 ? 1 : 48 / tiles;
   if (s > kb) s = kb;
   if (s < 1) s = 1;
   const int64_t per = (kb + s - 1) / s;
@@ -65,19 +68,27 @@ inline int permute_chunks(int T) { return (T + 255) / 256; }
 // Tile planner: routed groups (device offsets [G+1], rows <= n_rows) followed
 // by n_shared groups of T rows each (token rows 0..T-1 of the unpermuted
 // activations, output rows shared_o_row + s*T).  Heavy groups first.
+// Also writes the chunk prefix of the groups in plan order (grp_cp [n_grp + 1]), then
+// their prefix in half chunks (grp_cp[n_grp + 1 ..], n_grp + 1 entries), and the number
+// of groups (n_grp); the GEMM kernels use them to order their tiles.
 cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared, int T,
                         int shared_o_row, int chunk_rows, Chunk* chunks, int32_t* n_chunks,
-                        int* status, cudaStream_t s);
+                        int32_t* grp_cp, int32_t* n_grp, int* status, cudaStream_t s);
 
 enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4 };
 
 struct GemmLaunch {
   int mode;
-  // weight (A) maps per segment and token (B) maps per segment
+  int tile_tokens;           // bf16 expert GEMMs: token-tile width (32, 128 or 256)
+  bool halves;               // chunks are twice the tile width: one tile per half chunk
+  // weight (A) maps per segment; token (B) maps per segment with boxes of 128, 64,
+  // 32 and 16 rows
   CUtensorMap wmap[2];
-  CUtensorMap tmap[2];
+  CUtensorMap tmap[2][4];
   const Chunk* chunks;       // device (FFN modes)
   const int32_t* n_chunks;   // device (FFN modes)
+  const int32_t* grp_cp;     // device (FFN modes): plan-order group chunk prefix
+  const int32_t* n_grp;      // device (FFN modes)
   int router_T;              // router mode: tokens
   int n_mblk;                // 128-row weight blocks per group
   int k_blocks;              // K / 64 (bf16) or K / 128 (e4m3)

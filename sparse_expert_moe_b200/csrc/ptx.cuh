@@ -58,8 +58,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // (and the caller must stop) if the CTA abort flag is raised or the clock
 // budget runs out; in the latter case MOE_ERR_TIMEOUT goes to *status and the
 // abort flag is raised for the other warps of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+__device__ __forceinline__ bool mbar_wait_budget(uint64_t* bar, uint32_t parity,
+                                                 volatile int* abort_flag, int* status,
+                                                 long long budget_cycles) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
@@ -67,13 +68,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 255u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitBudgetCycles) {
+      if (clock64() - t0 > budget_cycles) {
         record_status(status, kStatusTimeout);
         *abort_flag = 1;
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  return mbar_wait_budget(bar, parity, abort_flag, status, kWaitBudgetCycles);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -45,7 +45,15 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     float l = 0.f, kk = -FLT_MAX;
     if (e < E) {
       l = __ldg(row + e);
-      for (int q = 1; q < n_partials; ++q) l += __ldg(row + q * partial_stride + e);
+      int q = 1;
+      for (; q + 3 < n_partials; q += 4) {   // fixed order: ((l + p1) + p2) + p3) + p4 ...
+        const float a = __ldg(row + q * partial_stride + e);
+        const float b = __ldg(row + (q + 1) * partial_stride + e);
+        const float c = __ldg(row + (q + 2) * partial_stride + e);
+        const float d = __ldg(row + (q + 3) * partial_stride + e);
+        l = (((l + a) + b) + c) + d;
+      }
+      for (; q < n_partials; ++q) l += __ldg(row + q * partial_stride + e);
       if (score == 0) {
         kk = l;
       } else {

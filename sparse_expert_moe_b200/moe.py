@@ -71,6 +71,7 @@ def load_library() -> ctypes.CDLL:
                                      ctypes.POINTER(ctypes.c_void_p)],
         "moe_read_device_status": [P, P, ctypes.POINTER(ctypes.c_int)],
         "moe_reset_device_status": [P, P],
+        "moe_selftest_bounded_wait": [P, ctypes.c_longlong, P],
     }
     for name, argtypes in sigs.items():
         fn = getattr(lib, name)
@@ -204,6 +205,11 @@ def moe_read_device_status(ws, stream=None) -> int:
 
 def moe_reset_device_status(ws, stream=None):
     _check("moe_reset_device_status", load_library().moe_reset_device_status(_p(ws), _stream(stream)))
+
+
+def moe_selftest_bounded_wait(ws, budget_cycles, stream=None):
+    _check("moe_selftest_bounded_wait",
+           load_library().moe_selftest_bounded_wait(_p(ws), int(budget_cycles), _stream(stream)))
 
 
 def moe_status_string(code: int) -> str:

@@ -157,3 +157,18 @@ def test_permute_out_of_range_index_sets_device_status():
     assert inv_perm[5, 1] == -1 and inv_perm[9, 0] == -1
     moe.moe_reset_device_status(ws)
     assert moe.moe_read_device_status(ws) == 0
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait that nothing completes ends after its budget with MOE_ERR_TIMEOUT in the
+    status word (no trap, no hang), and the device keeps working afterwards."""
+    ws = torch.zeros(4096, dtype=torch.uint8, device=DEV)
+    moe.moe_selftest_bounded_wait(ws, 2_000_000)          # ~1 ms of SM clock
+    assert moe.moe_read_device_status(ws) == 6             # MOE_ERR_TIMEOUT
+    moe.moe_reset_device_status(ws)
+    assert moe.moe_read_device_status(ws) == 0
+    T, E, k = 16, 8, 2
+    L = margin_logits(T, E, k, "softmax", None, seed=3)
+    idx, _ = _route_gpu(moe.make_config(T, 128, E, k, 128, 0, score="softmax"), L, None)
+    ridx, _ = oracle.route(L.astype(np.float64), "softmax", k)
+    assert np.array_equal(idx, ridx)
