@@ -12,7 +12,8 @@
 //     offsets and per-(chunk, expert) base rows.
 //  2. rank: each CTA rebuilds its masks; the row of (token t, slot j) with
 //     expert e is base(chunk, e) + earlier warps' counts + popc(mask & lanes
-//     below t).
+//     below t).  With a single chunk (T <= 256) the count CTA, which still holds
+//     the masks after the scan, ranks the pairs itself (one launch less).
 //  3. gather: x_perm[r] = x[perm_token[r]], one warp per row, 16-byte vectors.
 #include <cuda_runtime.h>
 
@@ -50,8 +51,10 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __res
                                                             int T, int E, int k,
                                                             int32_t* __restrict__ chunk_counts,
                                                             int32_t* __restrict__ offsets,
-                                                            unsigned* done, int* status) {
-  extern __shared__ uint32_t masks[];   // [kWarps][E]
+                                                            unsigned* done, int* status,
+                                                            int32_t* __restrict__ perm_token,
+                                                            int32_t* __restrict__ inv_perm) {
+  extern __shared__ uint32_t masks[];   // [kWarps][E] (+ [kWarps][E] row bases, one chunk)
   __shared__ int32_t warp_tot[kWarps];
   __shared__ bool is_last;
   const int nch = gridDim.x;
@@ -113,6 +116,34 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __res
   }
   if (tid == blockDim.x - 1) offsets[E] = run;
   if (tid == 0) *done = 0u;   // ready for the next call on this workspace
+  if (nch == 1 && perm_token) {
+    // one chunk (T <= 256): this CTA still holds the lane masks, so it ranks the pairs
+    // itself instead of a second launch; chunk bases are the group offsets
+    __syncthreads();
+    int32_t* wbase = reinterpret_cast<int32_t*>(masks + kWarps * E);
+    for (int e = tid; e < E; e += blockDim.x) {
+      int r = __ldcg(offsets + e);
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        wbase[w * E + e] = r;
+        r += __popc(masks[w * E + e]);
+      }
+    }
+    __syncthreads();
+    const int t = threadIdx.x;
+    const uint32_t below = (1u << lane) - 1u;
+    if (t < T) {
+      for (int j = 0; j < k; ++j) {
+        const int e = __ldg(topk_idx + static_cast<size_t>(t) * k + j);
+        int row = -1;
+        if (e >= 0 && e < E) {
+          row = wbase[warp * E + e] + __popc(masks[warp * E + e] & below);
+          perm_token[row] = t;
+        }
+        inv_perm[static_cast<size_t>(t) * k + j] = row;
+      }
+    }
+  }
 }
 
 __global__ void __launch_bounds__(256) permute_rank_kernel(const int32_t* __restrict__ topk_idx,
@@ -203,10 +234,23 @@ cudaError_t launch_permute(const int32_t* topk_idx, int T, int E, int k, const v
                                static_cast<int>(smem_rank));
     if (err != cudaSuccess) return err;
   }
-  permute_count_kernel<<<nch, kChunkTokens, smem_count, s>>>(topk_idx, T, E, k, chunk_counts,
-                                                             offsets, done, status);
-  permute_rank_kernel<<<nch, kChunkTokens, smem_rank, s>>>(topk_idx, T, E, k, chunk_counts,
-                                                           perm_token, inv_perm);
+  if (nch == 1) {
+    // one chunk: the count kernel ranks too
+    if (smem_rank > 48 * 1024) {
+      err = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_rank));
+      if (err != cudaSuccess) return err;
+    }
+    permute_count_kernel<<<1, kChunkTokens, smem_rank, s>>>(topk_idx, T, E, k, chunk_counts,
+                                                            offsets, done, status, perm_token,
+                                                            inv_perm);
+  } else {
+    permute_count_kernel<<<nch, kChunkTokens, smem_count, s>>>(topk_idx, T, E, k, chunk_counts,
+                                                               offsets, done, status, nullptr,
+                                                               nullptr);
+    permute_rank_kernel<<<nch, kChunkTokens, smem_rank, s>>>(topk_idx, T, E, k, chunk_counts,
+                                                             perm_token, inv_perm);
+  }
   const int rows = T * k;
   int blocks = (rows + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;

@@ -123,8 +123,10 @@ cudaError_t launch_route(const float* logits, int n_partials, long long partial_
                          const float* sel_bias, int T, int E, int k, int score, int32_t* topk_idx,
                          float* topk_w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int threads = 256;
-  const int blocks = (T + 7) / 8;
+  // small batches: 2 warps per block so that the tokens spread over many SMs (the
+  // partial-logit loads are latency-bound)
+  const int threads = T >= 2048 ? 256 : 64;
+  const int blocks = (T + threads / 32 - 1) / (threads / 32);
   if (E <= 32)
     route_kernel<1><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
                                                k, score, topk_idx, topk_w);
