@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="profiling case: the workload with this many tokens T (with --experts)")
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling case: the workload with only this many routed experts "
                          "(drawn without the stored recipe; not a bench line)")
@@ -150,9 +152,23 @@ def work_model(spec, offsets):
     ffn1_flops = 2.0 * rows * 2 * I * d
     ffn2_flops = 2.0 * rows * I * d
     layer_flops = 2.0 * rows * 3 * I * d + 2.0 * T * d * E
+    # per-expert operands of the two GEMMs: each expert (group of n > 0 rows) is bound by
+    # its own flops or by its own bytes (weights once, its rows in, h out and in, y out)
+    n_all = np.concatenate([sizes[sizes > 0], np.full(S, T)]).astype(np.float64)
+    group_flops = 2.0 * n_all * 3 * I * d
+    group_bytes = 3.0 * I * d * wb + n_all * (d * ab + 2 * I * 2 + d * 2)
     return dict(touched=touched, ffn1_bytes=ffn1_bytes, ffn2_bytes=ffn2_bytes,
                 layer_weight_bytes=layer_weight_bytes, ffn1_flops=ffn1_flops,
-                ffn2_flops=ffn2_flops, layer_flops=layer_flops)
+                ffn2_flops=ffn2_flops, layer_flops=layer_flops,
+                group_flops=group_flops, group_bytes=group_bytes)
+
+
+def per_expert_bound_ms(wm, tflops, gbs):
+    """Sum over experts of max(flops / tensor peak, bytes / HBM peak) for the two expert
+    GEMMs: the time they take when every expert runs at its own roofline and experts do
+    not overlap one another's HBM and tensor phases."""
+    t = np.maximum(wm["group_flops"] / (tflops * 1e12), wm["group_bytes"] / (gbs * 1e9))
+    return float(t.sum() * 1e3)
 
 
 def bound_of(name):
@@ -364,6 +380,8 @@ def run_ours(args):
     if args.experts:
         from dataclasses import replace
         spec = replace(inputs.SPECS[name], E=args.experts)
+        if args.tokens:
+            spec = replace(spec, T=args.tokens)
         wl = inputs.make_workload(spec, 0)
     else:
         wl = inputs.load_workload(name)
@@ -458,6 +476,9 @@ def run_ours(args):
             peak *= 2.0   # nominal fp8 : bf16 ratio of the dense tensor-core peaks
         unit = "TFLOP/s"
         units_note = "2 * (T*k + S*T) * 2I * d"
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * \
+        (2.0 if spec.weight == "e4m3" else 1.0)
+    ffn_bound_ms = per_expert_bound_ms(wm, tensor_peak, peaks["hbm_gbs"])
     tokens = spec.T * world
     value = replica_throughput(spec.T, world, ms_total, K)
     line = {
@@ -465,7 +486,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if spec.weight == "e4m3" else "bf16", "data": "synthetic",
-        "config": {"workload": name if not args.experts else f"{name} with E={spec.E} (profiling case)",
+        "config": {"workload": name if not args.experts else
+                   f"{name} with E={spec.E}, T={spec.T} (profiling case)",
                    "T": spec.T, "d_model": spec.d_model, "E": spec.E,
                    "top_k": spec.top_k, "d_ff": spec.d_ff, "n_shared": spec.n_shared,
                    "score": spec.score, "parallelism": f"replicas x{world}",
@@ -478,7 +500,9 @@ def run_ours(args):
         "layer": {"weight_bytes_touched": wm["layer_weight_bytes"],
                   "hbm_frac_layer": wm["layer_weight_bytes"] / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
                   "tflops_layer": wm["layer_flops"] / (ms_step * 1e-3) / 1e12,
-                  "touched_experts": wm["touched"]},
+                  "touched_experts": wm["touched"],
+                  "ffn_per_expert_bound_ms": ffn_bound_ms,
+                  "ffn_frac_of_per_expert_bound": ffn_bound_ms / (stage_ms["ffn1"] + stage_ms["ffn2"])},
         "stages_ms": stage_ms,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

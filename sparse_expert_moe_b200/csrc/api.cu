@@ -108,6 +108,12 @@ int bf16_chunk_rows(int64_t max_group) {
   return max_group <= kChunkRows ? kChunkRowsNarrow : kChunkRowsWide;
 }
 
+// FP8 chunk rows: 112, or 224 once groups can exceed 112 rows (FFN2 tiles of 224
+// tokens, FFN1 tiles of half a chunk).
+int fp8_chunk_rows(int64_t max_group) {
+  return max_group <= kChunkRowsFP8 ? kChunkRowsFP8 : 2 * kChunkRowsFP8;
+}
+
 // ---------------------------------------------------------------- TMA maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -188,7 +194,7 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
                        const uint4* wsf13_0, const uint4* wsf2_0, int64_t G0, const void* a1,
                        const uint32_t* a1_sf, int64_t a1_rows, const void* w13_1, const void* w2_1,
                        const uint4* wsf13_1, const uint4* wsf2_1, int64_t S, int64_t rows_all,
-                       void* y, cudaStream_t s, cudaEvent_t* ev = nullptr) {
+                       void* y, int chunk_rows, cudaStream_t s, cudaEvent_t* ev = nullptr) {
   const int64_t d = c.d_model, I = c.d_ff;
   void* h = at<void>(ws, L.h);
   uint32_t* h_sf = at<uint32_t>(ws, L.h_sf);
@@ -200,7 +206,10 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
   g.status = status_word(ws);
   g.num_sms = num_sms();
 
+  // FFN1 tiles hold 112 tokens (half a 224-row chunk when chunks are 224 rows); FFN2
+  // tiles are one chunk wide
   g.mode = kFFN1F8;
+  g.halves = chunk_rows == 2 * kChunkRowsFP8;
   if (!make_tmap_u8(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) || !make_tok_maps(g.tmap[0], a0, a0_rows, d, true))
     return MOE_ERR_CUDA;
   g.wsf[0] = wsf13_0;
@@ -237,6 +246,8 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
   g.mode = kFFN2F8;
+  g.halves = false;
+  g.tile_tokens = chunk_rows;
   if (!make_tmap_u8(&g.wmap[0], w2_0, G0 * d, I, 128) || !make_tok_maps(g.tmap[0], h, rows_all, I, true))
     return MOE_ERR_CUDA;
   g.wsf[0] = wsf2_0;
@@ -285,10 +296,12 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
   g.status = status_word(ws);
   g.num_sms = num_sms();
 
-  // FFN1 keeps 128-token tiles (two accumulator buffers overlap its SwiGLU epilogue with
-  // the next tile's MMAs); on 256-row chunks each tile takes half a chunk.  FFN2 runs
-  // 256-token tiles on them.
+  // FFN1 keeps single-CTA 128-token tiles (two accumulator buffers overlap its SwiGLU
+  // epilogue with the next tile's MMAs); on 256-row chunks each tile takes half a chunk.
+  // FFN2 runs tiles one chunk wide, on 256-row chunks as CTA pairs (tcgen05
+  // cta_group::2: 256 output columns x 256 tokens per pair tile).
   g.mode = kFFN1;
+  g.pair = false;
   g.tile_tokens = chunk_rows == kChunkRowsWide ? kChunkRows : chunk_rows;
   g.halves = chunk_rows == kChunkRowsWide;
   if (!make_tmap_bf16(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) ||
@@ -314,6 +327,7 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
   g.mode = kFFN2;
+  g.pair = chunk_rows == kChunkRowsWide && d % 256 == 0;   // pair tiles: 256 output columns
   g.tile_tokens = chunk_rows;
   g.halves = false;
   if (!make_tmap_bf16(&g.wmap[0], w2_0, G0 * d, I, 128) ||
@@ -325,7 +339,7 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
     g.wmap[1] = g.wmap[0];
   }
   copy_maps(g.tmap[1], g.tmap[0]);
-  g.n_mblk = static_cast<int>(d / 128);
+  g.n_mblk = static_cast<int>(g.pair ? d / 256 : d / 128);
   g.k_blocks = static_cast<int>(I / 64);
   g.w_rows_per_group = static_cast<int>(d);
   g.up_offset = 0;
@@ -437,13 +451,14 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
       st = cuda_status(launch_weight_sf(w2_s, static_cast<size_t>(n_groups) * (d / 128) * (I / 128),
                                         wsf2, stream));
     if (st == MOE_OK)
-      st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRowsFP8,
+      st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, fp8_chunk_rows(n_rows),
                                    at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
                                at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
                                    status_word(ws), stream));
     if (st != MOE_OK) return st;
     return run_ffn_fp8(*cfg, L, ws, a, a_sf, n_rows, w13, w2, wsf13, wsf2, n_groups, nullptr,
-                       nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0, n_rows, y, stream);
+                       nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0, n_rows, y,
+                       fp8_chunk_rows(n_rows), stream);
   }
   const int chunk_rows = bf16_chunk_rows(n_rows);
   st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, chunk_rows,
@@ -598,7 +613,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
 
   // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs.  Groups hold at
   // most T rows, which picks the bf16 token-tile width.
-  const int chunk_rows = fp8 ? kChunkRowsFP8 : bf16_chunk_rows(T);
+  const int chunk_rows = fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T);
   st = cuda_status(launch_plan(offsets, c.E, static_cast<int>(R), c.n_shared, c.T,
                                static_cast<int>(R), chunk_rows,
                                at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
@@ -611,7 +626,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
     const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
     const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
     st = run_ffn_fp8(c, L, ws, x_perm, x_perm_sf, R, w13_b, w2_b, wsf13, wsf2, E, x_b, x_sf, T, ws13_b,
-                     ws2_b, wsf13 + E * n13, wsf2 + E * n2, S, L.rows_all, y_rows, s,
+                     ws2_b, wsf13 + E * n13, wsf2 + E * n2, S, L.rows_all, y_rows, chunk_rows, s,
                      ev ? ev + 5 : nullptr);
   } else {
     st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows,

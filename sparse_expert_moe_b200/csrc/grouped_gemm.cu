@@ -46,9 +46,11 @@ constexpr uint32_t kABytes = kBM * kRowBytes;
 constexpr uint32_t kSFAtomBytes = 512;    // 128 rows x 4 UE8M0 bytes (tcgen05.cp 32x128b source)
 
 constexpr int kTokBoxes = 4;              // token boxes of 128, 64, 32, 16 rows
+constexpr uint32_t kMaxSmem = 227 * 1024;  // opt-in dynamic shared memory per CTA
+constexpr int kRingSlots = 16;            // stage barriers of a byte ring
 
 struct DevParams {
-  CUtensorMap wmap[2];
+  CUtensorMap wmap[2];        // weight maps per segment (boxes of 128 rows)
   CUtensorMap tmap[2][kTokBoxes];
   const Chunk* chunks;
   const int32_t* n_chunks;
@@ -87,18 +89,22 @@ template <int MODE, int NTW = kChunkRows>
 struct Cfg {
   static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8;
   static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8;   // gate + up accumulators
-  static_assert(NTW == kChunkRows || !(kFP8 || MODE == kRouter), "tile width: bf16 expert GEMMs");
+  static_assert(NTW == kChunkRows || MODE != kRouter, "router tiles are 128 tokens wide");
   static constexpr int kATiles = kGLU ? 2 : 1;
-  static constexpr int kNT = kFP8 ? kChunkRowsFP8 : NTW;
+  // FP8 tiles: 112 tokens (112 / 224 are passed in as NTW), leaving TMEM room for the
+  // per-stage scale factors
+  static constexpr int kNT = (kFP8 && NTW == kChunkRows) ? kChunkRowsFP8 : NTW;
+  static constexpr int kSFBAtoms = (kNT + 127) / 128;               // 128 token rows per atom
   static constexpr int kAccBufs = (kGLU && kNT > 128) ? 1 : 2;
   static constexpr uint32_t kBBytes = kNT * kRowBytes;
-  static constexpr uint32_t kSFBytes = kFP8 ? (kATiles + 1) * kSFAtomBytes : 0;
+  static constexpr uint32_t kSFBytes = kFP8 ? (kATiles + kSFBAtoms) * kSFAtomBytes : 0;
   static constexpr uint32_t kStageBytes =
       ((kATiles * kABytes + kBBytes + kSFBytes + 1023) / 1024) * 1024;
   static constexpr int kStagesFit = static_cast<int>((192u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
   static constexpr uint32_t kAccCols = kGLU ? 2 * kNT : kNT;        // per accumulator buffer
-  static constexpr uint32_t kSFColsPerStage = 16;                     // <= 3 atoms x 4 columns
+  static constexpr uint32_t kSFColsPerStage = 16;                     // <= 4 atoms x 4 columns
+  static_assert(!kFP8 || (kATiles + kSFBAtoms) * 4 <= 16, "scale atoms per stage");
   static constexpr uint32_t kSFCols = kFP8 ? kStages * kSFColsPerStage : 0;
   static constexpr uint32_t kColsUsed = kAccBufs * kAccCols + kSFCols;
   static constexpr uint32_t kTmemCols =
@@ -107,8 +113,16 @@ struct Cfg {
   static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;      // per epilogue warp: 16 x 32 x 4 B
   static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;   // group (half-)chunk prefixes
   static constexpr uint32_t kRedBytes = kFP8 ? 2 * 4 * 128 * 4 : 0;  // FP8 amax exchange
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + kStagingBytes +
-                                         kGrpBytes + 16 + kRedBytes + 1024 /*align*/;
+  // Stage ring: FP8 keeps fixed stages (the scale warp and the per-stage TMEM scale
+  // columns are indexed by stage); bf16 stages take their actual size out of a byte ring
+  // filling the rest of shared memory.
+  static constexpr uint32_t kFixedBytes = 1024 /*barriers*/ + kStagingBytes + kGrpBytes + 16 +
+                                          kRedBytes + 1024 /*align*/;
+  static constexpr int kSlots = kFP8 ? kStages : kRingSlots;
+  static constexpr uint32_t kRingBytes =
+      kFP8 ? kStages * kStageBytes : ((kMaxSmem - kFixedBytes) / 1024) * 1024;
+  static constexpr uint32_t kSmemBytes = kRingBytes + kFixedBytes;
+  static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
   static_assert(kColsUsed <= 512, "TMEM budget");
 };
 
@@ -201,6 +215,51 @@ __device__ __forceinline__ int e4m3_scale_exponent(uint32_t amax_bits) {
   return max(-127, min(127, e));
 }
 
+// Pipeline stages of variable size in a byte ring of shared memory.  A stage takes the
+// bytes right after the previous stage's, or offset 0 when it would run past the end of
+// the ring, so a tile of few tokens keeps more K blocks of weights in flight than a tile
+// of many.  The MMA thread releases stages in issue order, so the bytes in flight are
+// those between the end of the released prefix and the head (counted mod 2^32, skipped
+// ring tails included).  The producer thread keeps the counters in registers and each
+// slot's end in shared memory (`end`); the consumer learns each stage's offset from
+// `slot_off`, written before the stage's full-barrier arrive.
+template <int kSlots, uint32_t kRing>
+struct StageRing {
+  uint32_t head = 0;       // bytes reserved so far, mod 2^32 (skipped tails included)
+  uint32_t pos = 0;        // ring offset of the head
+  uint32_t freed = 0;      // end of the released prefix, same count as head
+  uint32_t issued = 0, released = 0;
+  uint32_t* end;           // [kSlots] shared memory: each slot's end, same count as head
+
+  // Reserves `bytes` (a multiple of 1024, at most kRing) for the next stage, waiting on
+  // the empty barriers of the oldest stages as needed; false if a wait ran out.
+  __device__ __forceinline__ bool acquire(uint32_t bytes, uint64_t* empty_bar,
+                                          volatile int* abort_flag, int* status, uint32_t& slot,
+                                          uint32_t& off) {
+    uint32_t skip = 0;
+    off = pos;
+    if (off + bytes > kRing) {                          // skip the ring's tail
+      skip = kRing - off;
+      off = 0;
+    }
+    // [off, off + bytes) is free once at most this many bytes before it are in flight
+    const int32_t allowed = max(0, static_cast<int32_t>(kRing - bytes - skip));
+    while (issued - released >= static_cast<uint32_t>(kSlots) ||
+           static_cast<int32_t>(head - freed) > allowed) {
+      const uint32_t s = released % kSlots;
+      if (!mbar_wait(&empty_bar[s], (released / kSlots) & 1u, abort_flag, status)) return false;
+      freed = end[s];
+      ++released;
+    }
+    slot = issued % kSlots;
+    head += skip + bytes;
+    pos = off + bytes;
+    end[slot] = head;
+    ++issued;
+    return true;
+  }
+};
+
 // Writes a warp's 16 (rows) x 32 (columns) output block: each lane holds one column's
 // 16 values; they pass through the warp's shared-memory staging area so that global
 // memory sees 16-byte vector stores (each row's 32 elements are contiguous), rows at
@@ -232,14 +291,16 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  uint64_t* empty_bar = full_bar + C::kStages;
-  uint64_t* tfull_bar = empty_bar + C::kStages;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
+  uint64_t* empty_bar = full_bar + C::kSlots;
+  uint64_t* tfull_bar = empty_bar + C::kSlots;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* red_bar = tempty_bar + 2;                            // [2] FP8 amax exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint8_t* staging = smem + C::kStages * C::kStageBytes + 1024;  // [4 warps][16 x 32 x 4 B]
+  uint32_t* slot_off = tmem_slot + 2;                            // [kSlots] stage offsets
+  uint32_t* slot_end = slot_off + C::kSlots;                     // [kSlots] producer's ring state
+  uint8_t* staging = smem + C::kRingBytes + 1024;                // [4 warps][16 x 32 x 4 B]
   int32_t* grp_cp = reinterpret_cast<int32_t*>(staging + C::kStagingBytes);
   // FP8: [2 buffers][4 warps][128 tokens] per-warp amax of the tile's h values
   uint32_t* red = reinterpret_cast<uint32_t*>(staging + C::kStagingBytes + C::kGrpBytes + 16);
@@ -248,7 +309,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
+    for (int i = 0; i < C::kSlots; ++i) {
       mbar_init(&full_bar[i], C::kFP8 ? 1 + 32 : 1);
       mbar_init(&empty_bar[i], 1);
     }
@@ -283,7 +344,8 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
+      StageRing<C::kSlots, C::kRingBytes> ring;
+      ring.end = slot_end;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
@@ -294,30 +356,29 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
         const int n_pad = (c.nrows + 15) & ~15;
         // the second GEMM reads the h rows the first one wrote (output numbering)
         const int tok_row = (MODE == kFFN2 || MODE == kFFN2F8) ? c.o_row : c.b_row;
-        const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;
+        const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;   // TMA bytes per stage
+        const uint32_t stage_bytes = C::kFP8 ? C::kStageBytes : bytes;     // ring bytes per stage
         const CUtensorMap* wm = &p.wmap[c.seg];
         for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) {
+          uint32_t slot, soff;
+          if (!ring.acquire(stage_bytes, empty_bar, abort_flag, p.status, slot, soff)) {
             ok = false;
             break;
           }
-          uint8_t* st = tiles + stage * C::kStageBytes;
+          uint8_t* st = tiles + soff;
+          slot_off[slot] = soff;
           const int kx = kb * (C::kFP8 ? 128 : 64);   // element coordinate of this K block
-          mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          tma_load_2d(st, wm, &full_bar[stage], kx, a_row);
-          if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[stage], kx, a_row + p.up_offset);
+          mbar_arrive_expect_tx(&full_bar[slot], bytes);
+          tma_load_2d(st, wm, &full_bar[slot], kx, a_row);
+          if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[slot], kx, a_row + p.up_offset);
           uint8_t* bt = st + C::kATiles * kABytes;
           // token rows as boxes of 128 / 64 / 32 / 16 rows covering n_pad
           for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
             const int rows = 128 >> bi;
             while (n_pad - off >= rows) {
-              tma_load_2d(bt + off * kRowBytes, &p.tmap[c.seg][bi], &full_bar[stage], kx, tok_row + off);
+              tma_load_2d(bt + off * kRowBytes, &p.tmap[c.seg][bi], &full_bar[slot], kx, tok_row + off);
               off += rows;
             }
-          }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
           }
         }
       }
@@ -347,7 +408,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_u32(tiles + stage * C::kStageBytes);
+          const uint32_t st = smem_u32(tiles) + slot_off[stage];
           const uint32_t bt = st + C::kATiles * kABytes;
           if (C::kFP8) {
             // scale factors of this stage: smem (written by the scale warp) -> TMEM
@@ -357,7 +418,11 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
             const uint32_t sfb = sfa + C::kATiles * 4;
             tmem_cp_32x128b_warpx4(sfa, smem_desc_noswizzle(sf_smem));
             if (C::kGLU) tmem_cp_32x128b_warpx4(sfa + 4, smem_desc_noswizzle(sf_smem + kSFAtomBytes));
-            tmem_cp_32x128b_warpx4(sfb, smem_desc_noswizzle(sf_smem + C::kATiles * kSFAtomBytes));
+            // token-side scales: one atom per 128 token rows, in consecutive 4-column groups
+#pragma unroll
+            for (int a = 0; a < C::kSFBAtoms; ++a)
+              tmem_cp_32x128b_warpx4(sfb + 4 * a,
+                                     smem_desc_noswizzle(sf_smem + (C::kATiles + a) * kSFAtomBytes));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
@@ -377,7 +442,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
             }
           }
           umma_commit(&empty_bar[stage]);
-          if (++stage == C::kStages) {
+          if (++stage == C::kSlots) {
             stage = 0;
             phase ^= 1u;
           }
@@ -519,11 +584,12 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           cp_async_16(sf + kSFAtomBytes + lane * 16, wsf + static_cast<size_t>(up_rb + mb) * p.k_blocks + kb);
         uint8_t* sfb = sf + C::kATiles * kSFAtomBytes;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int n = lane + 32 * j;
+        for (int j = 0; j < 4 * C::kSFBAtoms; ++j) {
+          const int n = lane + 32 * j;     // atom j / 4, in-atom row group j % 4
           if (n < n_pad) {
             const int row = min(tok_row + n, trows - 1);
-            cp_async_4(sfb + lane * 16 + j * 4, tsf + static_cast<size_t>(kb) * tld + row);
+            cp_async_4(sfb + (j >> 2) * kSFAtomBytes + lane * 16 + (j & 3) * 4,
+                       tsf + static_cast<size_t>(kb) * tld + row);
           }
         }
         cp_async_mbar_arrive_noinc(&full_bar[stage]);
@@ -540,6 +606,197 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------- CTA-pair kernel
+// The bf16 second GEMM on 256 x 256 UMMA tiles shared by the two CTAs of a cluster
+// (tcgen05 cta_group::2): tile = 256 output columns x up to 256 tokens; CTA r stages W2
+// rows 128r..128r+127 and half of the tile's tokens, so every byte a CTA loads feeds
+// twice the flops of a single-CTA 128-row tile.  Roles as in grouped_gemm_kernel; the
+// leader CTA (rank 0) issues the MMAs and owns the full and accumulator-empty barriers
+// that both CTAs' loads and epilogues signal; the MMA commits arrive on both CTAs'
+// empty and accumulator-full barriers (multicast commit).
+struct PairCfg {
+  static constexpr int kNT = kChunkRowsWide;              // tokens per tile (both CTAs)
+  static constexpr uint32_t kAccCols = kNT;               // 256 fp32 columns per buffer
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;
+  static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;
+  static constexpr uint32_t kFixedBytes =
+      1024 /*barriers*/ + kStagingBytes + kGrpBytes + 16 + 1024 /*align*/;
+  // stages: 128 weight rows + up to 128 token rows each, out of a byte ring (StageRing)
+  static constexpr int kSlots = kRingSlots;
+  static constexpr uint32_t kRingBytes = ((kMaxSmem - kFixedBytes) / 1024) * 1024;
+  static constexpr uint32_t kSmemBytes = kRingBytes + kFixedBytes;
+  static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    pair_ffn2_kernel(const __grid_constant__ DevParams p) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
+  uint64_t* empty_bar = full_bar + C::kSlots;
+  uint64_t* tfull_bar = empty_bar + C::kSlots;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* slot_off = tmem_slot + 2;                    // [kSlots] stage offsets
+  uint32_t* slot_end = slot_off + C::kSlots;             // [kSlots] producer's ring state
+  uint8_t* staging = smem + C::kRingBytes + 1024;
+  int32_t* grp_cp = reinterpret_cast<int32_t*>(staging + C::kStagingBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kSlots; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 2 * 128);               // both CTAs' epilogue threads
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.wmap[0]);
+    tma_prefetch_desc(&p.tmap[0][0]);
+  }
+  const int n_grp = *p.n_grp;
+  for (int i = threadIdx.x; i < 2 * (n_grp + 1); i += blockDim.x) grp_cp[i] = p.grp_cp[i];
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int n_tiles = *p.n_chunks * p.n_mblk;
+  const int cl = blockIdx.x >> 1, n_cl = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      // both CTAs reserve the same sizes in the same order: equal offsets
+      StageRing<C::kSlots, C::kRingBytes> ring;
+      ring.end = slot_end;
+      bool ok = true;
+      for (int t = cl; t < n_tiles && ok; t += n_cl) {
+        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+        const Chunk c = get_chunk<kFFN2>(p, tc.chunk);
+        const int n_pad = (c.nrows + 31) & ~31;         // N: each CTA holds N / 2 token rows
+        const int half = n_pad >> 1;
+        const int tok_row = c.o_row + static_cast<int>(rank) * half;
+        const int a_row = c.group * p.w_rows_per_group + tc.mb * 256 + static_cast<int>(rank) * 128;
+        const CUtensorMap* wm = &p.wmap[c.seg];
+        const uint32_t stage_bytes = kABytes + half * kRowBytes;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          uint32_t slot, soff;
+          if (!ring.acquire(stage_bytes, empty_bar, abort_flag, p.status, slot, soff)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = tiles + soff;
+          slot_off[slot] = soff;
+          const uint32_t bar = mapa_shared(&full_bar[slot], 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2 * kABytes + n_pad * kRowBytes);
+          const int kx = kb * 64;
+          tma_load_2d_pair(st, wm, bar, kx, a_row);
+          uint8_t* bt = st + kABytes;
+          for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
+            const int rows = 128 >> bi;
+            while (half - off >= rows) {
+              tma_load_2d_pair(bt + off * kRowBytes, &p.tmap[c.seg][bi], bar, kx, tok_row + off);
+              off += rows;
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = cl; t < n_tiles && ok; t += n_cl, ++it) {
+        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+        const Chunk c = get_chunk<kFFN2>(p, tc.chunk);
+        const int n_pad = (c.nrows + 31) & ~31;
+        const uint32_t idesc = idesc_bf16_f32(256, n_pad);
+        const uint32_t acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * C::kAccCols;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(tiles) + slot_off[stage];
+          const uint32_t bt = st + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_pair(d0, umma_desc_sw128(st + kk * 32), umma_desc_sw128(bt + kk * 32), idesc,
+                           (kb | kk) ? 1u : 0u);
+          umma_commit_pair(&empty_bar[stage], 0x3);
+          if (++stage == C::kSlots) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit_pair(&tfull_bar[acc], 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    // CTA r's TMEM lanes are its 128 output columns; columns of TMEM are the tile's tokens
+    const int sub = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(&tempty_bar[0], 0);
+    const uint32_t tempty_leader1 = mapa_shared(&tempty_bar[1], 0);
+    int it = 0;
+    for (int t = cl; t < n_tiles; t += n_cl, ++it) {
+      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+      const Chunk c = get_chunk<kFFN2>(p, tc.chunk);
+      const uint32_t acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + acc * C::kAccCols;
+      const int col0 = tc.mb * 256 + static_cast<int>(rank) * 128 + sub * 32;
+      for (int n0 = 0; n0 < c.nrows; n0 += 16) {
+        float v[16];
+        tmem_ld16(tb + n0, v);
+        __nv_bfloat16 yv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v[i]);
+        store_block_16x32(static_cast<__nv_bfloat16*>(p.out) +
+                              static_cast<size_t>(c.o_row + n0) * p.ld_out + col0,
+                          p.ld_out, c.nrows - n0, yv,
+                          reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, C::kTmemCols);
 }
 
 // ---------------------------------------------------------------- planner
@@ -671,8 +928,7 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   using C = Cfg<MODE, NTW>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
   DevParams p;
-  p.wmap[0] = g.wmap[0];
-  p.wmap[1] = g.wmap[1];
+  for (int i = 0; i < 2; ++i) p.wmap[i] = g.wmap[i];
   for (int i = 0; i < 2; ++i)
     for (int j = 0; j < kTokBoxes; ++j) p.tmap[i][j] = g.tmap[i][j];
   p.chunks = g.chunks;
@@ -715,7 +971,51 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+static cudaError_t launch_pair_ffn2(const GemmLaunch& g, cudaStream_t s) {
+  using C = PairCfg;
+  DevParams p;
+  for (int i = 0; i < 2; ++i) p.wmap[i] = g.wmap[i];
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < kTokBoxes; ++j) p.tmap[i][j] = g.tmap[i][j];
+  p.chunks = g.chunks;
+  p.n_chunks = g.n_chunks;
+  p.grp_cp = g.grp_cp;
+  p.n_grp = g.n_grp;
+  p.halves = 0;
+  p.router_T = 0;
+  p.n_mblk = g.n_mblk;
+  p.k_blocks = g.k_blocks;
+  p.k_splits = 1;
+  p.k_per_split = g.k_blocks;
+  p.split_stride = 0;
+  p.w_rows_per_group = g.w_rows_per_group;
+  p.up_offset = g.up_offset;
+  p.m_valid = g.m_valid;
+  p.out = g.out;
+  p.ld_out = g.ld_out;
+  p.status = g.status;
+  cudaError_t err = cudaFuncSetAttribute(pair_ffn2_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::kSmemBytes));
+  if (err != cudaSuccess) return err;
+  // persistent: as many clusters as can be resident at once (a GPC with an odd number of
+  // free SMs leaves one idle), so that no cluster waits for another to finish
+  int grid = g.num_sms & ~1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(192);
+  lc.dynamicSmemBytes = C::kSmemBytes;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, pair_ffn2_kernel, &lc) == cudaSuccess &&
+      clusters > 0 && 2 * clusters < grid)
+    grid = 2 * clusters;
+  (void)cudaGetLastError();
+  pair_ffn2_kernel<<<grid, 192, C::kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
+  if (g.pair) return g.mode == kFFN2 ? launch_pair_ffn2(g, s) : cudaErrorInvalidValue;
   switch (g.mode) {
     case kRouter: return launch_mode<kRouter, kChunkRows>(g, s);
     case kFFN1:
@@ -726,7 +1026,9 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
       if (g.tile_tokens == kChunkRowsWide) return launch_mode<kFFN2, kChunkRowsWide>(g, s);
       return launch_mode<kFFN2, kChunkRows>(g, s);
     case kFFN1F8: return launch_mode<kFFN1F8, kChunkRows>(g, s);
-    case kFFN2F8: return launch_mode<kFFN2F8, kChunkRows>(g, s);
+    case kFFN2F8:
+      if (g.tile_tokens == 2 * kChunkRowsFP8) return launch_mode<kFFN2F8, 2 * kChunkRowsFP8>(g, s);
+      return launch_mode<kFFN2F8, kChunkRows>(g, s);
     default: return cudaErrorInvalidValue;
   }
 }

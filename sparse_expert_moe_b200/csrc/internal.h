@@ -80,9 +80,10 @@ enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4 };
 struct GemmLaunch {
   int mode;
   int tile_tokens;           // bf16 expert GEMMs: token-tile width (32, 128 or 256)
+  bool pair;                 // bf16 FFN2 on 256-token chunks: CTA-pair (cta_group::2) tiles
   bool halves;               // chunks are twice the tile width: one tile per half chunk
-  // weight (A) maps per segment; token (B) maps per segment with boxes of 128, 64,
-  // 32 and 16 rows
+  // weight (A) maps per segment (boxes of 128 rows); token (B) maps per segment with
+  // boxes of 128, 64, 32 and 16 rows
   CUtensorMap wmap[2];
   CUtensorMap tmap[2][4];
   const Chunk* chunks;       // device (FFN modes)

@@ -42,25 +42,36 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = i * 32 + lane;
-    float l = 0.f, kk = -FLT_MAX;
-    if (e < E) {
-      l = __ldg(row + e);
-      int q = 1;
-      for (; q + 3 < n_partials; q += 4) {   // fixed order: ((l + p1) + p2) + p3) + p4 ...
-        const float a = __ldg(row + q * partial_stride + e);
-        const float b = __ldg(row + (q + 1) * partial_stride + e);
-        const float c = __ldg(row + (q + 2) * partial_stride + e);
-        const float d = __ldg(row + (q + 3) * partial_stride + e);
-        l = (((l + a) + b) + c) + d;
-      }
-      for (; q < n_partials; ++q) l += __ldg(row + q * partial_stride + e);
-      if (score == 0) {
-        kk = l;
-      } else {
-        kk = sigmoidf_(l) + (sel_bias ? __ldg(sel_bias + e) : 0.f);
-      }
+    lg[i] = e < E ? __ldg(row + e) : 0.f;
+  }
+  // partial logits of a split-K router: all of a lane's values advance together, four
+  // partials at a time (4 * VPL independent loads in flight), each value summed in the
+  // fixed order p0 + p1 + p2 + ...
+  int q = 1;
+  for (; q + 3 < n_partials; q += 4) {
+    float a[VPL][4];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        a[i][u] = e < E ? __ldg(row + (q + u) * partial_stride + e) : 0.f;
     }
-    lg[i] = l;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) lg[i] = (((lg[i] + a[i][0]) + a[i][1]) + a[i][2]) + a[i][3];
+  }
+  for (; q < n_partials; ++q) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E) lg[i] += __ldg(row + q * partial_stride + e);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    float kk = -FLT_MAX;
+    if (e < E) kk = score == 0 ? lg[i] : sigmoidf_(lg[i]) + (sel_bias ? __ldg(sel_bias + e) : 0.f);
     key[i] = kk;
   }
 
