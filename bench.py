@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling case: the workload with only this many routed experts "
                          "(drawn without the stored recipe; not a bench line)")
+    ap.add_argument("--fp8-peak", action="store_true",
+                    help="measure the dense e4m3 GEMM peak (cuBLASLt) on cuda:0, print it, exit")
     return ap.parse_args()
 
 
@@ -64,6 +66,56 @@ def load_peaks():
         return p, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+FP8_PEAK_FILE = os.path.join(ROOT, "profiles", "fp8_peak.md")
+
+
+def load_fp8_peak():
+    """Dense e4m3 GEMM throughput measured on this machine's B200s (``bench.py --fp8-peak``,
+    recorded in profiles/fp8_peak.md as ``fp8_tflops_sustained: X``), else None."""
+    try:
+        for line in open(FP8_PEAK_FILE):
+            if line.startswith("fp8_tflops_sustained:"):
+                return float(line.split(":", 1)[1])
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def measure_fp8_peak(dev, n=8192, seconds=4.0):
+    """cuBLASLt e4m3 x e4m3 -> bf16 GEMM (torch._scaled_mm) n^3: best of 10 (burst) and a
+    back-to-back loop of `seconds` (sustained), 2 n^3 flops each."""
+    import torch
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    one = torch.ones((), device=dev)
+
+    def mm():
+        return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+    for _ in range(3):
+        mm()
+    torch.cuda.synchronize(dev)
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    iters = max(1, int(seconds * 1e3 / best))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        mm()
+    e1.record()
+    e1.synchronize()
+    flops = 2.0 * n ** 3
+    return {"fp8_tflops": flops / (best * 1e-3) / 1e12,
+            "fp8_tflops_sustained": flops / (e0.elapsed_time(e1) / iters * 1e-3) / 1e12,
+            "n": n, "iters": iters, "how": "torch._scaled_mm e4m3 x e4m3 -> bf16, unit scales"}
 
 
 def blas_threads():
@@ -473,11 +525,17 @@ def run_ours(args):
         achieved = wm["ffn1_flops"] / (stage_ms["ffn1"] * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         if spec.weight == "e4m3":
-            peak *= 2.0   # nominal fp8 : bf16 ratio of the dense tensor-core peaks
+            fp8 = load_fp8_peak()
+            if fp8 is not None:
+                peak, peak_src = fp8, "measured e4m3 (profiles/fp8_peak.md)"
+            else:
+                peak *= 2.0   # nominal fp8 : bf16 ratio of the dense tensor-core peaks
+                peak_src += " bf16 x 2 (nominal fp8 ratio)"
         unit = "TFLOP/s"
         units_note = "2 * (T*k + S*T) * 2I * d"
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * \
-        (2.0 if spec.weight == "e4m3" else 1.0)
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    if spec.weight == "e4m3":
+        tensor_peak = load_fp8_peak() or 2.0 * tensor_peak
     ffn_bound_ms = per_expert_bound_ms(wm, tensor_peak, peaks["hbm_gbs"])
     tokens = spec.T * world
     value = replica_throughput(spec.T, world, ms_total, K)
@@ -523,6 +581,9 @@ def run_ours(args):
 
 def main():
     args = parse()
+    if args.fp8_peak:
+        print(json.dumps(measure_fp8_peak("cuda:0")), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
