@@ -215,6 +215,22 @@ def work_model(spec, offsets):
                 group_flops=group_flops, group_bytes=group_bytes)
 
 
+def small_stage_bytes(spec):
+    """Algorithmic HBM bytes of the bandwidth-bound stages around the expert GEMMs (reads +
+    writes each stage must make at least once)."""
+    T, d, E, k, S = spec.T, spec.d_model, spec.E, spec.top_k, spec.n_shared
+    ab = 1 if spec.act == "e4m3" else 2
+    xs = 4 * (d // 128) if spec.act == "e4m3" else 0          # per-row activation scales
+    ob = 4 if spec.out == "f32" else 2
+    R = T * k
+    return {
+        "router_gemm": T * d * 2 + E * d * 2 + T * E * 4,
+        "route": T * E * 4 + (E * 4 if spec.score == "sigmoid_bias" else 0) + R * 8,
+        "permute": R * 4 + T * (d * ab + xs) + R * (d * ab + xs) + R * 8 + (E + 1) * 4,
+        "combine": (R + S * T) * d * 2 + R * 8 + T * d * ob,
+    }
+
+
 def per_expert_bound_ms(wm, tflops, gbs):
     """Sum over experts of max(flops / tensor peak, bytes / HBM peak) for the two expert
     GEMMs: the time they take when every expert runs at its own roofline and experts do
@@ -562,6 +578,9 @@ def run_ours(args):
                   "ffn_per_expert_bound_ms": ffn_bound_ms,
                   "ffn_frac_of_per_expert_bound": ffn_bound_ms / (stage_ms["ffn1"] + stage_ms["ffn2"])},
         "stages_ms": stage_ms,
+        "stages_hbm": {n: {"bytes": int(v), "gbs": v / (stage_ms[n] * 1e-3) / 1e9,
+                           "frac": v / (stage_ms[n] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                       for n, v in small_stage_bytes(spec).items()},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": LAUNCHES_PER_STEP * K,

@@ -44,12 +44,13 @@ cudaError_t launch_route(const float* logits, int n_partials, long long partial_
 
 // K splits of the router GEMM for T tokens, E experts and d_model: about 48 CTAs
 // when the (token chunk, expert block) tiles alone are fewer -- enough to stream
-// Wr quickly, few enough that summing the partial logits stays cheap; every split
-// non-empty.  Host only.
+// Wr quickly, few enough that summing the partial logits stays cheap (at most 32, the
+// route kernel's limit); every split non-empty.  Host only.
 inline int router_splits(int64_t T, int64_t E, int64_t d) {
   const int64_t tiles = ((T + 127) / 128) * ((E + 127) / 128);
   const int64_t kb = d / 64;
   int64_t s = tiles >= 48 ? 1 : 48 / tiles;
+  if (s > 32) s = 32;
   if (s > kb) s = kb;
   if (s < 1) s = 1;
   const int64_t per = (kb + s - 1) / s;

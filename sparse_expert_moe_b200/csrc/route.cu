@@ -6,8 +6,8 @@
 // bias routing" ("Chapter 7: Serving Mega MoE at scale").
 //
 // Each lane holds experts lane, lane+32, ... of the token's logit row (coalesced
-// 128-byte loads); when the router GEMM split K across CTAs, the partial logits
-// are summed here in a fixed order, so repeated runs are bit-identical.  k rounds
+// 128-byte loads); when the router GEMM split K across CTAs, a CTA per token first
+// sums the partial logits in a fixed order, so repeated runs are bit-identical.  k rounds
 // of a warp-wide arg-max (shuffle butterfly; key descending, equal keys to the
 // lower expert index) pick the slots in order; lane j keeps slot j and computes
 // its gate with one more butterfly.  HBM-bound: the kernel reads
@@ -27,46 +27,14 @@ __device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
+// Top-k of one token's logits, held by one warp (lane: experts lane, lane + 32, ...), and
+// the gates of the selected experts; lanes 0..k-1 write slot `lane`.
 template <int VPL>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int n_partials,
-                                                    long long partial_stride,
-                                                    const float* __restrict__ sel_bias, int T, int E,
-                                                    int k, int score, int32_t* __restrict__ topk_idx,
-                                                    float* __restrict__ topk_w) {
-  const int token = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (token >= T) return;
-  const float* row = logits + static_cast<size_t>(token) * E;
-
-  float key[VPL], lg[VPL];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int e = i * 32 + lane;
-    lg[i] = e < E ? __ldg(row + e) : 0.f;
-  }
-  // partial logits of a split-K router: all of a lane's values advance together, four
-  // partials at a time (4 * VPL independent loads in flight), each value summed in the
-  // fixed order p0 + p1 + p2 + ...
-  int q = 1;
-  for (; q + 3 < n_partials; q += 4) {
-    float a[VPL][4];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = i * 32 + lane;
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        a[i][u] = e < E ? __ldg(row + (q + u) * partial_stride + e) : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) lg[i] = (((lg[i] + a[i][0]) + a[i][1]) + a[i][2]) + a[i][3];
-  }
-  for (; q < n_partials; ++q) {
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E) lg[i] += __ldg(row + q * partial_stride + e);
-    }
-  }
+__device__ __forceinline__ void select_and_gate(const float (&lg)[VPL], int lane, int E, int k,
+                                                int score, const float* __restrict__ sel_bias,
+                                                int token, int32_t* __restrict__ topk_idx,
+                                                float* __restrict__ topk_w) {
+  float key[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = i * 32 + lane;
@@ -128,35 +96,92 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   }
 }
 
+// One warp per token on complete logits (n_partials == 1).
+template <int VPL>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
+                                                    const float* __restrict__ sel_bias, int T, int E,
+                                                    int k, int score, int32_t* __restrict__ topk_idx,
+                                                    float* __restrict__ topk_w) {
+  const int token = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (token >= T) return;
+  const float* row = logits + static_cast<size_t>(token) * E;
+  float lg[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    lg[i] = e < E ? __ldg(row + e) : 0.f;
+  }
+  select_and_gate<VPL>(lg, lane, E, k, score, sel_bias, token, topk_idx, topk_w);
+}
+
+// One CTA per token on the partial logits of a split-K router: thread t sums the partials
+// of experts t, t + 256, ... in the fixed order p0 + p1 + p2 + ... (all of a thread's loads
+// in flight together: one round of latency instead of one per few partials), the sums go
+// through shared memory, and warp 0 selects.
+template <int VPL>
+__global__ void __launch_bounds__(256) route_partials_kernel(const float* __restrict__ logits,
+                                                             int n_partials, long long partial_stride,
+                                                             const float* __restrict__ sel_bias,
+                                                             int T, int E, int k, int score,
+                                                             int32_t* __restrict__ topk_idx,
+                                                             float* __restrict__ topk_w) {
+  constexpr int kMaxPartials = 32;
+  __shared__ float sums[32 * VPL];
+  const int token = blockIdx.x;
+  const float* row = logits + static_cast<size_t>(token) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float v[kMaxPartials];
+#pragma unroll
+    for (int q = 0; q < kMaxPartials; ++q)
+      v[q] = q < n_partials ? __ldg(row + q * partial_stride + e) : 0.f;
+    float l = v[0];
+#pragma unroll
+    for (int q = 1; q < kMaxPartials; ++q)
+      if (q < n_partials) l += v[q];
+    sums[e] = l;
+  }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  float lg[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    lg[i] = e < E ? sums[e] : 0.f;
+  }
+  select_and_gate<VPL>(lg, lane, E, k, score, sel_bias, token, topk_idx, topk_w);
+}
+
+template <int VPL>
+cudaError_t launch_route_vpl(const float* logits, int n_partials, long long partial_stride,
+                             const float* sel_bias, int T, int E, int k, int score,
+                             int32_t* topk_idx, float* topk_w, cudaStream_t s) {
+  if (n_partials > 1) {
+    route_partials_kernel<VPL><<<T, 256, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T,
+                                                 E, k, score, topk_idx, topk_w);
+  } else {
+    // small batches: 2 warps per block so that the tokens spread over many SMs
+    const int threads = T >= 2048 ? 256 : 64;
+    const int blocks = (T + threads / 32 - 1) / (threads / 32);
+    route_kernel<VPL><<<blocks, threads, 0, s>>>(logits, sel_bias, T, E, k, score, topk_idx, topk_w);
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_route(const float* logits, int n_partials, long long partial_stride,
                          const float* sel_bias, int T, int E, int k, int score, int32_t* topk_idx,
                          float* topk_w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  // small batches: 2 warps per block so that the tokens spread over many SMs (the
-  // partial-logit loads are latency-bound)
-  const int threads = T >= 2048 ? 256 : 64;
-  const int blocks = (T + threads / 32 - 1) / (threads / 32);
-  if (E <= 32)
-    route_kernel<1><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
-                                               k, score, topk_idx, topk_w);
-  else if (E <= 64)
-    route_kernel<2><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
-                                               k, score, topk_idx, topk_w);
-  else if (E <= 128)
-    route_kernel<4><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
-                                               k, score, topk_idx, topk_w);
-  else if (E <= 256)
-    route_kernel<8><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
-                                               k, score, topk_idx, topk_w);
-  else if (E <= 512)
-    route_kernel<16><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
-                                               k, score, topk_idx, topk_w);
-  else
-    route_kernel<32><<<blocks, threads, 0, s>>>(logits, n_partials, partial_stride, sel_bias, T, E,
-                                               k, score, topk_idx, topk_w);
-  return cudaGetLastError();
+  if (n_partials < 1 || n_partials > 32) return cudaErrorInvalidValue;
+  if (E <= 32) return launch_route_vpl<1>(logits, n_partials, partial_stride, sel_bias, T, E, k, score, topk_idx, topk_w, s);
+  if (E <= 64) return launch_route_vpl<2>(logits, n_partials, partial_stride, sel_bias, T, E, k, score, topk_idx, topk_w, s);
+  if (E <= 128) return launch_route_vpl<4>(logits, n_partials, partial_stride, sel_bias, T, E, k, score, topk_idx, topk_w, s);
+  if (E <= 256) return launch_route_vpl<8>(logits, n_partials, partial_stride, sel_bias, T, E, k, score, topk_idx, topk_w, s);
+  if (E <= 512) return launch_route_vpl<16>(logits, n_partials, partial_stride, sel_bias, T, E, k, score, topk_idx, topk_w, s);
+  return launch_route_vpl<32>(logits, n_partials, partial_stride, sel_bias, T, E, k, score, topk_idx, topk_w, s);
 }
 
 }  // namespace moe

@@ -34,3 +34,14 @@ def test_per_expert_bound_reduces_to_each_side():
     # a bound never below either total divided by its own peak
     b = bench.per_expert_bound_ms(wm, 1.0, 1.0)
     assert b >= max(wm["group_flops"].sum() / 1e12, wm["group_bytes"].sum() / 1e9) * 1e3
+
+
+def test_small_stage_bytes_prefill_shape():
+    """R1 prefill: the permutation reads x once and writes T k rows; the combine reads the
+    T k routed rows and T shared rows and writes T rows (d = 7168, bf16)."""
+    spec = inputs.SPECS["r1_prefill"]
+    b = bench.small_stage_bytes(spec)
+    T, d, k = 8192, 7168, 8
+    assert b["permute"] == pytest.approx(T * d * 2 * (1 + k), rel=1e-3)
+    assert b["combine"] == pytest.approx((T * k + T) * d * 2 + T * d * 2, rel=1e-3)
+    assert b["route"] == pytest.approx(T * 256 * 4, rel=0.1)
