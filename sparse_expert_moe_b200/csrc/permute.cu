@@ -179,7 +179,11 @@ __global__ void __launch_bounds__(256) permute_rank_kernel(const int32_t* __rest
   }
 }
 
-// One warp per permuted row; rows past offsets[E] (dropped pairs) are skipped.
+// One warp per permuted row; rows past offsets[E] (dropped pairs) are skipped.  x is
+// read k times (from L2 when it stays there) and x_perm is written once and not read
+// again by this kernel, so the stores are streaming (evict-first): the T k rows passing
+// through L2 on their way to HBM would otherwise push x out and turn its re-reads into
+// DRAM reads.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, int vec_per_row,
                                                           const float* __restrict__ x_scale,
                                                           int scale_cols, uint4* __restrict__ x_perm,
@@ -197,12 +201,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     for (; v + 96 < vec_per_row; v += 128) {
       const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), c = __ldg(src + v + 64),
                   d = __ldg(src + v + 96);
-      dst[v] = a;
-      dst[v + 32] = b;
-      dst[v + 64] = c;
-      dst[v + 96] = d;
+      __stcs(dst + v, a);
+      __stcs(dst + v + 32, b);
+      __stcs(dst + v + 64, c);
+      __stcs(dst + v + 96, d);
     }
-    for (; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+    for (; v < vec_per_row; v += 32) __stcs(dst + v, __ldg(src + v));
     if (x_scale)
       for (int c = lane; c < scale_cols; c += 32)
         x_perm_scale[static_cast<size_t>(r) * scale_cols + c] =
