@@ -101,9 +101,8 @@ moe_status check_config(const moe_config* c) {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// bf16 chunk rows (= token-tile width of the expert GEMMs) for groups of at most
-// `max_group` rows: 32 for decode-sized batches, else 256 (FFN2 tiles of 256 tokens,
-// FFN1 tiles of half a chunk).
+// bf16 chunk rows for groups of at most `max_group` rows: 32 for decode-sized batches
+// (one token tile per chunk), else 256 (expert GEMM tiles of half a chunk).
 int bf16_chunk_rows(int64_t max_group) {
   return max_group <= kChunkRows ? kChunkRowsNarrow : kChunkRowsWide;
 }
@@ -298,10 +297,9 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
 
   // FFN1 keeps single-CTA 128-token tiles (two accumulator buffers overlap its SwiGLU
   // epilogue with the next tile's MMAs); on 256-row chunks each tile takes half a chunk.
-  // FFN2 runs tiles one chunk wide, on 256-row chunks as CTA pairs (tcgen05
-  // cta_group::2: 256 output columns x 256 tokens per pair tile).
+  // FFN2 does the same with 256 output columns per tile (two 128-row weight blocks per
+  // stage) when d_model allows it, else one 128-row block on whole chunks.
   g.mode = kFFN1;
-  g.pair = false;
   g.tile_tokens = chunk_rows == kChunkRowsWide ? kChunkRows : chunk_rows;
   g.halves = chunk_rows == kChunkRowsWide;
   if (!make_tmap_bf16(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) ||
@@ -326,10 +324,10 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
-  g.mode = kFFN2;
-  g.pair = chunk_rows == kChunkRowsWide && d % 256 == 0;   // pair tiles: 256 output columns
-  g.tile_tokens = chunk_rows;
-  g.halves = false;
+  const bool m256 = d % 256 == 0;
+  g.mode = m256 ? kFFN2M256 : kFFN2;
+  g.halves = m256 && chunk_rows == kChunkRowsWide;
+  g.tile_tokens = g.halves ? kChunkRows : chunk_rows;
   if (!make_tmap_bf16(&g.wmap[0], w2_0, G0 * d, I, 128) ||
       !make_tok_maps(g.tmap[0], h, rows_all, I, false))
     return MOE_ERR_CUDA;
@@ -339,7 +337,7 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
     g.wmap[1] = g.wmap[0];
   }
   copy_maps(g.tmap[1], g.tmap[0]);
-  g.n_mblk = static_cast<int>(g.pair ? d / 256 : d / 128);
+  g.n_mblk = static_cast<int>(m256 ? d / 256 : d / 128);
   g.k_blocks = static_cast<int>(I / 64);
   g.w_rows_per_group = static_cast<int>(d);
   g.up_offset = 0;

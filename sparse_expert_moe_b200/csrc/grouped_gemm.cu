@@ -19,7 +19,11 @@
 // almost all of every MMA; with tokens on N the same kernel streams weights
 // at N = 16 and reaches full 128x128 tiles on heavy prefill groups.  FFN1 keeps
 // two accumulators per tile (gate rows and up rows of the same h columns), so
-// SiLU(gate) * up happens in registers and h is written once.
+// SiLU(gate) * up happens in registers and h is written once.  FFN2 likewise
+// stages two 128-row weight blocks per K block (256 output columns, two
+// accumulators): every stage then carries 32 KB of weights, as in FFN1, which the
+// weight stream needs to reach the HBM roofline (one 16 KB block per stage left
+// FFN2 at 77-91% of it).
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one lane)       -- fills a STAGES-deep smem ring
@@ -27,9 +31,8 @@
 //   warps 2..5  epilogue: TMEM -> registers -> global (warp w reads TMEM lanes
 //               32*(w%4)..+31, the sub-partition it may access)
 // Two TMEM accumulator buffers let the epilogue of tile i overlap the MMAs of
-// tile i+1.  Tiles are (chunk, 128-row weight block), weight block fastest, so
-// CTAs running at the same time share a chunk's token rows through L2.
-// Chunks come from the planner below, largest groups first.
+// tile i+1.  Tiles are (token chunk, weight block) laid out group by group (see
+// tile_coord); chunks come from the planner below, largest groups first.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -80,17 +83,20 @@ struct DevParams {
   int ld_out_sf;
 };
 
-// NTW: token-tile width of the bf16 expert GEMMs.  128 by default; 32 for decode-sized
-// batches (small shared-memory token tiles leave room for a deeper weight ring: 5 / 9
-// stages); 256 for large groups (twice the reuse of every weight byte loaded into
-// shared memory; a 256-wide FFN1 would hold its gate and up accumulators in all 512
-// TMEM columns -- one buffer -- so FFN1 instead takes half a 256-row chunk per tile).
+// NTW: token-tile width of the bf16 expert GEMMs.  128 by default -- half of a 256-row
+// chunk once groups can exceed 128 rows (a 256-wide tile with two accumulators, gate
+// and up or two output blocks, would need all 512 TMEM columns for one buffer, and its
+// epilogue could no longer hide behind the next tile's MMAs); 32 for decode-sized
+// batches (small token tiles leave shared memory to a deeper weight ring); 256 only for
+// the single-block FFN2 used when d_model is not a multiple of 256.
 template <int MODE, int NTW = kChunkRows>
 struct Cfg {
   static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8;
   static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8;   // gate + up accumulators
+  static constexpr bool kM256 = MODE == kFFN2M256;                  // two output blocks
+  static constexpr bool kSecondA = kGLU || kM256;                   // two weight tiles per stage
   static_assert(NTW == kChunkRows || MODE != kRouter, "router tiles are 128 tokens wide");
-  static constexpr int kATiles = kGLU ? 2 : 1;
+  static constexpr int kATiles = kSecondA ? 2 : 1;
   // FP8 tiles: 112 tokens (112 / 224 are passed in as NTW), leaving TMEM room for the
   // per-stage scale factors
   static constexpr int kNT = (kFP8 && NTW == kChunkRows) ? kChunkRowsFP8 : NTW;
@@ -102,7 +108,7 @@ struct Cfg {
       ((kATiles * kABytes + kBBytes + kSFBytes + 1023) / 1024) * 1024;
   static constexpr int kStagesFit = static_cast<int>((192u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
-  static constexpr uint32_t kAccCols = kGLU ? 2 * kNT : kNT;        // per accumulator buffer
+  static constexpr uint32_t kAccCols = kSecondA ? 2 * kNT : kNT;    // per accumulator buffer
   static constexpr uint32_t kSFColsPerStage = 16;                     // <= 4 atoms x 4 columns
   static_assert(!kFP8 || (kATiles + kSFBAtoms) * 4 <= 16, "scale atoms per stage");
   static constexpr uint32_t kSFCols = kFP8 ? kStages * kSFColsPerStage : 0;
@@ -191,15 +197,16 @@ __device__ __forceinline__ TileCoord tile_coord(const DevParams& p, int t, const
 
 // The rows a tile covers: its chunk, or one half of it when chunks are twice the
 // tile width (nrows <= 0: nothing to do -- every role skips the tile alike).
-template <int MODE>
+template <int MODE, int NTW>
 __device__ __forceinline__ Chunk tile_rows(const DevParams& p, const TileCoord& tc) {
   Chunk c = get_chunk<MODE>(p, tc.chunk);
   if (p.halves) {
-    const int off = tc.half * Cfg<MODE>::kNT;
+    constexpr int kNT = Cfg<MODE, NTW>::kNT;
+    const int off = tc.half * kNT;
     c.b_row += off;
     c.o_row += off;
     c.nrows -= off;
-    if (c.nrows > Cfg<MODE>::kNT) c.nrows = Cfg<MODE>::kNT;
+    if (c.nrows > kNT) c.nrows = kNT;
   }
   return c;
 }
@@ -349,13 +356,16 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-        const Chunk c = tile_rows<MODE>(p, tc);
+        const Chunk c = tile_rows<MODE, NTW>(p, tc);
         if (c.nrows <= 0) continue;
         const int mb = tc.mb;
-        const int a_row = c.group * p.w_rows_per_group + mb * kBM;
+        // first weight row of the tile; the second weight tile (FFN1: the up rows of the
+        // same h columns; FFN2 M256: the next 128 output columns) starts a_row2
+        const int a_row = c.group * p.w_rows_per_group + mb * kBM * (C::kM256 ? 2 : 1);
+        const int a_row2 = a_row + (C::kGLU ? p.up_offset : kBM);
         const int n_pad = (c.nrows + 15) & ~15;
         // the second GEMM reads the h rows the first one wrote (output numbering)
-        const int tok_row = (MODE == kFFN2 || MODE == kFFN2F8) ? c.o_row : c.b_row;
+        const int tok_row = (MODE == kFFN2 || MODE == kFFN2M256 || MODE == kFFN2F8) ? c.o_row : c.b_row;
         const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;   // TMA bytes per stage
         const uint32_t stage_bytes = C::kFP8 ? C::kStageBytes : bytes;     // ring bytes per stage
         const CUtensorMap* wm = &p.wmap[c.seg];
@@ -370,7 +380,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           const int kx = kb * (C::kFP8 ? 128 : 64);   // element coordinate of this K block
           mbar_arrive_expect_tx(&full_bar[slot], bytes);
           tma_load_2d(st, wm, &full_bar[slot], kx, a_row);
-          if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[slot], kx, a_row + p.up_offset);
+          if (C::kSecondA) tma_load_2d(st + kABytes, wm, &full_bar[slot], kx, a_row2);
           uint8_t* bt = st + C::kATiles * kABytes;
           // token rows as boxes of 128 / 64 / 32 / 16 rows covering n_pad
           for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-        const Chunk c = tile_rows<MODE>(p, tc);
+        const Chunk c = tile_rows<MODE, NTW>(p, tc);
         if (c.nrows <= 0) continue;
         const int n_pad = (c.nrows + 15) & ~15;
         const uint32_t idesc = C::kFP8 ? idesc_e4m3_bs(kBM, n_pad) : idesc_bf16_f32(kBM, n_pad);
@@ -438,7 +448,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
               const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
               const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
               umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, accum);
-              if (C::kGLU) umma_bf16(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, accum);
+              if (C::kSecondA) umma_bf16(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, accum);
             }
           }
           umma_commit(&empty_bar[stage]);
@@ -461,7 +471,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
     bool epi_ok = true;
     for (int t = blockIdx.x; t < n_tiles && epi_ok; t += gridDim.x) {
       const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-      const Chunk c = tile_rows<MODE>(p, tc);
+      const Chunk c = tile_rows<MODE, NTW>(p, tc);
       if (c.nrows <= 0) continue;
       const int mb = tc.mb;
       const uint32_t acc = it % C::kAccBufs;
@@ -528,6 +538,21 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
                                 static_cast<size_t>(c.o_row + n0) * p.ld_out + (m - lane),
                             p.ld_out, c.nrows - n0, hv,
                             reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+        } else if (MODE == kFFN2M256) {
+          // accumulator j holds output columns mb * 256 + j * 128 + (0..127)
+          float v0[16], v1[16];
+          tmem_ld16x2(tb + n0, tb + C::kNT + n0, v0, v1);
+          __nv_bfloat16 yv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v0[i]);
+          __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
+                                (mb * 2 * kBM + m_local - lane);
+          store_block_16x32(yrow, p.ld_out, c.nrows - n0, yv,
+                            reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v1[i]);
+          store_block_16x32(yrow + kBM, p.ld_out, c.nrows - n0, yv,
+                            reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
         } else if (MODE == kFFN2 || MODE == kFFN2F8) {
           float v[16];
           tmem_ld16(tb + n0, v);
@@ -564,7 +589,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
     const int up_rb = p.up_offset / kBM;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
       const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-      const Chunk c = tile_rows<MODE>(p, tc);
+      const Chunk c = tile_rows<MODE, NTW>(p, tc);
       if (c.nrows <= 0) continue;
       const int mb = tc.mb;
       const int n_pad = (c.nrows + 15) & ~15;
@@ -606,197 +631,6 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
-}
-
-// ---------------------------------------------------------------- CTA-pair kernel
-// The bf16 second GEMM on 256 x 256 UMMA tiles shared by the two CTAs of a cluster
-// (tcgen05 cta_group::2): tile = 256 output columns x up to 256 tokens; CTA r stages W2
-// rows 128r..128r+127 and half of the tile's tokens, so every byte a CTA loads feeds
-// twice the flops of a single-CTA 128-row tile.  Roles as in grouped_gemm_kernel; the
-// leader CTA (rank 0) issues the MMAs and owns the full and accumulator-empty barriers
-// that both CTAs' loads and epilogues signal; the MMA commits arrive on both CTAs'
-// empty and accumulator-full barriers (multicast commit).
-struct PairCfg {
-  static constexpr int kNT = kChunkRowsWide;              // tokens per tile (both CTAs)
-  static constexpr uint32_t kAccCols = kNT;               // 256 fp32 columns per buffer
-  static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;
-  static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;
-  static constexpr uint32_t kFixedBytes =
-      1024 /*barriers*/ + kStagingBytes + kGrpBytes + 16 + 1024 /*align*/;
-  // stages: 128 weight rows + up to 128 token rows each, out of a byte ring (StageRing)
-  static constexpr int kSlots = kRingSlots;
-  static constexpr uint32_t kRingBytes = ((kMaxSmem - kFixedBytes) / 1024) * 1024;
-  static constexpr uint32_t kSmemBytes = kRingBytes + kFixedBytes;
-  static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
-};
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    pair_ffn2_kernel(const __grid_constant__ DevParams p) {
-  using C = PairCfg;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* tiles = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
-  uint64_t* empty_bar = full_bar + C::kSlots;
-  uint64_t* tfull_bar = empty_bar + C::kSlots;
-  uint64_t* tempty_bar = tfull_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* slot_off = tmem_slot + 2;                    // [kSlots] stage offsets
-  uint32_t* slot_end = slot_off + C::kSlots;             // [kSlots] producer's ring state
-  uint8_t* staging = smem + C::kRingBytes + 1024;
-  int32_t* grp_cp = reinterpret_cast<int32_t*>(staging + C::kStagingBytes);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kSlots; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 2 * 128);               // both CTAs' epilogue threads
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&p.wmap[0]);
-    tma_prefetch_desc(&p.tmap[0][0]);
-  }
-  const int n_grp = *p.n_grp;
-  for (int i = threadIdx.x; i < 2 * (n_grp + 1); i += blockDim.x) grp_cp[i] = p.grp_cp[i];
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, C::kTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  const int n_tiles = *p.n_chunks * p.n_mblk;
-  const int cl = blockIdx.x >> 1, n_cl = gridDim.x >> 1;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      // both CTAs reserve the same sizes in the same order: equal offsets
-      StageRing<C::kSlots, C::kRingBytes> ring;
-      ring.end = slot_end;
-      bool ok = true;
-      for (int t = cl; t < n_tiles && ok; t += n_cl) {
-        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-        const Chunk c = get_chunk<kFFN2>(p, tc.chunk);
-        const int n_pad = (c.nrows + 31) & ~31;         // N: each CTA holds N / 2 token rows
-        const int half = n_pad >> 1;
-        const int tok_row = c.o_row + static_cast<int>(rank) * half;
-        const int a_row = c.group * p.w_rows_per_group + tc.mb * 256 + static_cast<int>(rank) * 128;
-        const CUtensorMap* wm = &p.wmap[c.seg];
-        const uint32_t stage_bytes = kABytes + half * kRowBytes;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
-          uint32_t slot, soff;
-          if (!ring.acquire(stage_bytes, empty_bar, abort_flag, p.status, slot, soff)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = tiles + soff;
-          slot_off[slot] = soff;
-          const uint32_t bar = mapa_shared(&full_bar[slot], 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2 * kABytes + n_pad * kRowBytes);
-          const int kx = kb * 64;
-          tma_load_2d_pair(st, wm, bar, kx, a_row);
-          uint8_t* bt = st + kABytes;
-          for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
-            const int rows = 128 >> bi;
-            while (half - off >= rows) {
-              tma_load_2d_pair(bt + off * kRowBytes, &p.tmap[c.seg][bi], bar, kx, tok_row + off);
-              off += rows;
-            }
-          }
-        }
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
-    if (lane == 0 && leader) {
-      uint32_t stage = 0, phase = 0;
-      bool ok = true;
-      int it = 0;
-      for (int t = cl; t < n_tiles && ok; t += n_cl, ++it) {
-        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-        const Chunk c = get_chunk<kFFN2>(p, tc.chunk);
-        const int n_pad = (c.nrows + 31) & ~31;
-        const uint32_t idesc = idesc_bf16_f32(256, n_pad);
-        const uint32_t acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
-        tc_fence_after();
-        const uint32_t d0 = tmem_base + acc * C::kAccCols;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = smem_u32(tiles) + slot_off[stage];
-          const uint32_t bt = st + kABytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_pair(d0, umma_desc_sw128(st + kk * 32), umma_desc_sw128(bt + kk * 32), idesc,
-                           (kb | kk) ? 1u : 0u);
-          umma_commit_pair(&empty_bar[stage], 0x3);
-          if (++stage == C::kSlots) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (ok) umma_commit_pair(&tfull_bar[acc], 0x3);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    // CTA r's TMEM lanes are its 128 output columns; columns of TMEM are the tile's tokens
-    const int sub = warp & 3;
-    const uint32_t tempty_leader0 = mapa_shared(&tempty_bar[0], 0);
-    const uint32_t tempty_leader1 = mapa_shared(&tempty_bar[1], 0);
-    int it = 0;
-    for (int t = cl; t < n_tiles; t += n_cl, ++it) {
-      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-      const Chunk c = get_chunk<kFFN2>(p, tc.chunk);
-      const uint32_t acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
-      bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + acc * C::kAccCols;
-      const int col0 = tc.mb * 256 + static_cast<int>(rank) * 128 + sub * 32;
-      for (int n0 = 0; n0 < c.nrows; n0 += 16) {
-        float v[16];
-        tmem_ld16(tb + n0, v);
-        __nv_bfloat16 yv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v[i]);
-        store_block_16x32(static_cast<__nv_bfloat16*>(p.out) +
-                              static_cast<size_t>(c.o_row + n0) * p.ld_out + col0,
-                          p.ld_out, c.nrows - n0, yv,
-                          reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
-      }
-      tc_fence_before();
-      mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-    }
-  }
-
-  tc_fence_before();
-  cluster_sync();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem_base, C::kTmemCols);
 }
 
 // ---------------------------------------------------------------- planner
@@ -971,60 +805,18 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-static cudaError_t launch_pair_ffn2(const GemmLaunch& g, cudaStream_t s) {
-  using C = PairCfg;
-  DevParams p;
-  for (int i = 0; i < 2; ++i) p.wmap[i] = g.wmap[i];
-  for (int i = 0; i < 2; ++i)
-    for (int j = 0; j < kTokBoxes; ++j) p.tmap[i][j] = g.tmap[i][j];
-  p.chunks = g.chunks;
-  p.n_chunks = g.n_chunks;
-  p.grp_cp = g.grp_cp;
-  p.n_grp = g.n_grp;
-  p.halves = 0;
-  p.router_T = 0;
-  p.n_mblk = g.n_mblk;
-  p.k_blocks = g.k_blocks;
-  p.k_splits = 1;
-  p.k_per_split = g.k_blocks;
-  p.split_stride = 0;
-  p.w_rows_per_group = g.w_rows_per_group;
-  p.up_offset = g.up_offset;
-  p.m_valid = g.m_valid;
-  p.out = g.out;
-  p.ld_out = g.ld_out;
-  p.status = g.status;
-  cudaError_t err = cudaFuncSetAttribute(pair_ffn2_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::kSmemBytes));
-  if (err != cudaSuccess) return err;
-  // persistent: as many clusters as can be resident at once (a GPC with an odd number of
-  // free SMs leaves one idle), so that no cluster waits for another to finish
-  int grid = g.num_sms & ~1;
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(grid);
-  lc.blockDim = dim3(192);
-  lc.dynamicSmemBytes = C::kSmemBytes;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, pair_ffn2_kernel, &lc) == cudaSuccess &&
-      clusters > 0 && 2 * clusters < grid)
-    grid = 2 * clusters;
-  (void)cudaGetLastError();
-  pair_ffn2_kernel<<<grid, 192, C::kSmemBytes, s>>>(p);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
-  if (g.pair) return g.mode == kFFN2 ? launch_pair_ffn2(g, s) : cudaErrorInvalidValue;
   switch (g.mode) {
     case kRouter: return launch_mode<kRouter, kChunkRows>(g, s);
     case kFFN1:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1, kChunkRowsNarrow>(g, s);
       return launch_mode<kFFN1, kChunkRows>(g, s);
-    case kFFN2:
+    case kFFN2M256:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2M256, kChunkRowsNarrow>(g, s);
+      return launch_mode<kFFN2M256, kChunkRows>(g, s);
+    case kFFN2:   // d_model not a multiple of 256: one 128-row weight block per tile
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2, kChunkRowsNarrow>(g, s);
-      if (g.tile_tokens == kChunkRowsWide) return launch_mode<kFFN2, kChunkRowsWide>(g, s);
-      return launch_mode<kFFN2, kChunkRows>(g, s);
+      return launch_mode<kFFN2, kChunkRowsWide>(g, s);
     case kFFN1F8: return launch_mode<kFFN1F8, kChunkRows>(g, s);
     case kFFN2F8:
       if (g.tile_tokens == 2 * kChunkRowsFP8) return launch_mode<kFFN2F8, 2 * kChunkRowsFP8>(g, s);

@@ -26,7 +26,8 @@ struct Chunk {
 
 constexpr int kChunkRows = 128;     // tokens per GEMM tile, bf16 (UMMA N <= 128)
 constexpr int kChunkRowsFP8 = 112;  // tokens per GEMM tile, FP8 (TMEM also holds scale factors)
-constexpr int kChunkRowsWide = 256; // tokens per GEMM tile, bf16 wide tiles (groups > 128 rows)
+constexpr int kChunkRowsWide = 256; // rows per chunk, bf16, once groups can exceed 128 rows
+                                    // (tiles take half a chunk)
 constexpr int kChunkRowsNarrow = 32; // tokens per GEMM tile, bf16 decode-sized batches
 constexpr int kMaxGroups = 1024 + 8;
 
@@ -76,12 +77,12 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
                         int shared_o_row, int chunk_rows, Chunk* chunks, int32_t* n_chunks,
                         int32_t* grp_cp, int32_t* n_grp, int* status, cudaStream_t s);
 
-enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4 };
+// kFFN2M256: FFN2 (bf16) with 256 weight rows per tile, as two 128-row blocks.
+enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5 };
 
 struct GemmLaunch {
   int mode;
   int tile_tokens;           // bf16 expert GEMMs: token-tile width (32, 128 or 256)
-  bool pair;                 // bf16 FFN2 on 256-token chunks: CTA-pair (cta_group::2) tiles
   bool halves;               // chunks are twice the tile width: one tile per half chunk
   // weight (A) maps per segment (boxes of 128 rows); token (B) maps per segment with
   // boxes of 128, 64, 32 and 16 rows
@@ -92,7 +93,7 @@ struct GemmLaunch {
   const int32_t* grp_cp;     // device (FFN modes): plan-order group chunk prefix
   const int32_t* n_grp;      // device (FFN modes)
   int router_T;              // router mode: tokens
-  int n_mblk;                // 128-row weight blocks per group
+  int n_mblk;                // weight-row tiles per group (128 rows; 256 for kFFN2M256)
   int k_blocks;              // K / 64 (bf16) or K / 128 (e4m3)
   int k_splits;              // router: K split across CTAs (1 = none); every split non-empty
   long long split_stride;    // router: elements between consecutive partial outputs
