@@ -297,8 +297,9 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
 
   // FFN1 keeps single-CTA 128-token tiles (two accumulator buffers overlap its SwiGLU
   // epilogue with the next tile's MMAs); on 256-row chunks each tile takes half a chunk.
-  // FFN2 does the same with 256 output columns per tile (two 128-row weight blocks per
-  // stage) when d_model allows it, else one 128-row block on whole chunks.
+  // FFN2 stages several 128-row weight blocks per K block (its tiles span 256 output
+  // columns, 512 on decode-sized token tiles), as d_model allows; with d_model not a
+  // multiple of 256, one 128-row block on whole chunks.
   g.mode = kFFN1;
   g.tile_tokens = chunk_rows == kChunkRowsWide ? kChunkRows : chunk_rows;
   g.halves = chunk_rows == kChunkRowsWide;
@@ -324,8 +325,9 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
-  const bool m256 = d % 256 == 0;
-  g.mode = m256 ? kFFN2M256 : kFFN2;
+  const bool m512 = d % 512 == 0 && chunk_rows == kChunkRowsNarrow;
+  const bool m256 = d % 256 == 0 && !m512;
+  g.mode = m512 ? kFFN2M512 : (m256 ? kFFN2M256 : kFFN2);
   g.halves = m256 && chunk_rows == kChunkRowsWide;
   g.tile_tokens = g.halves ? kChunkRows : chunk_rows;
   if (!make_tmap_bf16(&g.wmap[0], w2_0, G0 * d, I, 128) ||
@@ -337,7 +339,7 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
     g.wmap[1] = g.wmap[0];
   }
   copy_maps(g.tmap[1], g.tmap[0]);
-  g.n_mblk = static_cast<int>(m256 ? d / 256 : d / 128);
+  g.n_mblk = static_cast<int>(m512 ? d / 512 : (m256 ? d / 256 : d / 128));
   g.k_blocks = static_cast<int>(I / 64);
   g.w_rows_per_group = static_cast<int>(d);
   g.up_offset = 0;

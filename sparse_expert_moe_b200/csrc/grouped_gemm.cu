@@ -93,10 +93,10 @@ template <int MODE, int NTW = kChunkRows>
 struct Cfg {
   static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8;
   static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8;   // gate + up accumulators
-  static constexpr bool kM256 = MODE == kFFN2M256;                  // two output blocks
-  static constexpr bool kSecondA = kGLU || kM256;                   // two weight tiles per stage
+  // FFN2: 128-row weight blocks (= 128 output columns each) per tile
+  static constexpr int kOutBlocks = MODE == kFFN2M512 ? 4 : (MODE == kFFN2M256 ? 2 : 1);
   static_assert(NTW == kChunkRows || MODE != kRouter, "router tiles are 128 tokens wide");
-  static constexpr int kATiles = kSecondA ? 2 : 1;
+  static constexpr int kATiles = kGLU ? 2 : kOutBlocks;             // weight tiles per stage
   // FP8 tiles: 112 tokens (112 / 224 are passed in as NTW), leaving TMEM room for the
   // per-stage scale factors
   static constexpr int kNT = (kFP8 && NTW == kChunkRows) ? kChunkRowsFP8 : NTW;
@@ -108,7 +108,7 @@ struct Cfg {
       ((kATiles * kABytes + kBBytes + kSFBytes + 1023) / 1024) * 1024;
   static constexpr int kStagesFit = static_cast<int>((192u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
-  static constexpr uint32_t kAccCols = kSecondA ? 2 * kNT : kNT;    // per accumulator buffer
+  static constexpr uint32_t kAccCols = kATiles * kNT;               // per accumulator buffer
   static constexpr uint32_t kSFColsPerStage = 16;                     // <= 4 atoms x 4 columns
   static_assert(!kFP8 || (kATiles + kSFBAtoms) * 4 <= 16, "scale atoms per stage");
   static constexpr uint32_t kSFCols = kFP8 ? kStages * kSFColsPerStage : 0;
@@ -359,13 +359,13 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
         const Chunk c = tile_rows<MODE, NTW>(p, tc);
         if (c.nrows <= 0) continue;
         const int mb = tc.mb;
-        // first weight row of the tile; the second weight tile (FFN1: the up rows of the
-        // same h columns; FFN2 M256: the next 128 output columns) starts a_row2
-        const int a_row = c.group * p.w_rows_per_group + mb * kBM * (C::kM256 ? 2 : 1);
-        const int a_row2 = a_row + (C::kGLU ? p.up_offset : kBM);
+        // first weight row of the tile; FFN1's second weight tile holds the up rows of the
+        // same h columns, FFN2's further tiles the next 128-row blocks
+        const int a_row = c.group * p.w_rows_per_group + mb * kBM * C::kOutBlocks;
         const int n_pad = (c.nrows + 15) & ~15;
         // the second GEMM reads the h rows the first one wrote (output numbering)
-        const int tok_row = (MODE == kFFN2 || MODE == kFFN2M256 || MODE == kFFN2F8) ? c.o_row : c.b_row;
+        const int tok_row = (MODE == kFFN2 || MODE == kFFN2M256 || MODE == kFFN2M512 || MODE == kFFN2F8)
+                                ? c.o_row : c.b_row;
         const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;   // TMA bytes per stage
         const uint32_t stage_bytes = C::kFP8 ? C::kStageBytes : bytes;     // ring bytes per stage
         const CUtensorMap* wm = &p.wmap[c.seg];
@@ -380,7 +380,10 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           const int kx = kb * (C::kFP8 ? 128 : 64);   // element coordinate of this K block
           mbar_arrive_expect_tx(&full_bar[slot], bytes);
           tma_load_2d(st, wm, &full_bar[slot], kx, a_row);
-          if (C::kSecondA) tma_load_2d(st + kABytes, wm, &full_bar[slot], kx, a_row2);
+          if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[slot], kx, a_row + p.up_offset);
+#pragma unroll
+          for (int j = 1; j < C::kOutBlocks; ++j)
+            tma_load_2d(st + j * kABytes, wm, &full_bar[slot], kx, a_row + j * kBM);
           uint8_t* bt = st + C::kATiles * kABytes;
           // token rows as boxes of 128 / 64 / 32 / 16 rows covering n_pad
           for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
@@ -448,7 +451,9 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
               const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
               const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
               umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, accum);
-              if (C::kSecondA) umma_bf16(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, accum);
+#pragma unroll
+              for (int j = 1; j < C::kATiles; ++j)
+                umma_bf16(d0 + j * C::kNT, umma_desc_sw128(st + j * kABytes + kk * 32), bdesc, idesc, accum);
             }
           }
           umma_commit(&empty_bar[stage]);
@@ -538,21 +543,24 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
                                 static_cast<size_t>(c.o_row + n0) * p.ld_out + (m - lane),
                             p.ld_out, c.nrows - n0, hv,
                             reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
-        } else if (MODE == kFFN2M256) {
-          // accumulator j holds output columns mb * 256 + j * 128 + (0..127)
-          float v0[16], v1[16];
-          tmem_ld16x2(tb + n0, tb + C::kNT + n0, v0, v1);
-          __nv_bfloat16 yv[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v0[i]);
+        } else if (MODE == kFFN2M256 || MODE == kFFN2M512) {
+          // accumulator j holds output columns (mb * kOutBlocks + j) * 128 + (0..127)
           __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
-                                (mb * 2 * kBM + m_local - lane);
-          store_block_16x32(yrow, p.ld_out, c.nrows - n0, yv,
-                            reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+                                (mb * C::kOutBlocks * kBM + m_local - lane);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v1[i]);
-          store_block_16x32(yrow + kBM, p.ld_out, c.nrows - n0, yv,
-                            reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+          for (int j = 0; j < C::kOutBlocks; j += 2) {
+            float v0[16], v1[16];
+            tmem_ld16x2(tb + j * C::kNT + n0, tb + (j + 1) * C::kNT + n0, v0, v1);
+            __nv_bfloat16 yv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v0[i]);
+            store_block_16x32(yrow + j * kBM, p.ld_out, c.nrows - n0, yv,
+                              reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(v1[i]);
+            store_block_16x32(yrow + (j + 1) * kBM, p.ld_out, c.nrows - n0, yv,
+                              reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+          }
         } else if (MODE == kFFN2 || MODE == kFFN2F8) {
           float v[16];
           tmem_ld16(tb + n0, v);
@@ -814,6 +822,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
     case kFFN2M256:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2M256, kChunkRowsNarrow>(g, s);
       return launch_mode<kFFN2M256, kChunkRows>(g, s);
+    case kFFN2M512: return launch_mode<kFFN2M512, kChunkRowsNarrow>(g, s);
     case kFFN2:   // d_model not a multiple of 256: one 128-row weight block per tile
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2, kChunkRowsNarrow>(g, s);
       return launch_mode<kFFN2, kChunkRowsWide>(g, s);

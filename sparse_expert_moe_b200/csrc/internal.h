@@ -77,8 +77,10 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
                         int shared_o_row, int chunk_rows, Chunk* chunks, int32_t* n_chunks,
                         int32_t* grp_cp, int32_t* n_grp, int* status, cudaStream_t s);
 
-// kFFN2M256: FFN2 (bf16) with 256 weight rows per tile, as two 128-row blocks.
-enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5 };
+// kFFN2M256 / kFFN2M512: FFN2 (bf16) with 256 / 512 weight rows per tile, as two / four
+// 128-row blocks (M512: decode-sized token tiles only).
+enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5,
+                kFFN2M512 = 6 };
 
 struct GemmLaunch {
   int mode;

@@ -28,6 +28,7 @@ def _bf16(a):
     ([5, 0, 1, 130, 16, 17, 0, 128], 256, 256),     # ragged: empty, 1 row, > one 128-row chunk
     ([300], 128, 384),                               # one group, three chunks, ragged tail
     ([1, 1, 1, 1], 512, 128),
+    ([3, 0, 17, 32, 33], 1024, 256),                # decode-sized: 32-row chunks, 512-row weight tiles
 ])
 def test_grouped_ffn_vs_oracle(sizes, d, I):
     rng = np.random.default_rng(sum(sizes) + d + I)
@@ -135,6 +136,7 @@ def test_layer_tiny_config():
     (200, 384, 32, 8, 256, 2, "sigmoid_bias"),
     (130, 128, 1, 1, 128, 0, "softmax"),          # E = 1, k = 1: a dense SwiGLU FFN
     (520, 256, 4, 2, 128, 1, "sigmoid_bias"),     # heavy groups: several 128-row chunks each
+    (96, 1024, 16, 4, 256, 1, "sigmoid_bias"),    # decode-sized, two 512-row FFN2 weight tiles
 ])
 def test_layer_custom(T, d, E, k, I, S, score):
     spec = inputs.custom_spec(T, d, E, k, I, S, score=score)
