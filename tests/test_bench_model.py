@@ -45,3 +45,14 @@ def test_small_stage_bytes_prefill_shape():
     assert b["permute"] == pytest.approx(T * d * 2 * (1 + k), rel=1e-3)
     assert b["combine"] == pytest.approx((T * k + T) * d * 2 + T * d * 2, rel=1e-3)
     assert b["route"] == pytest.approx(T * 256 * 4, rel=0.1)
+
+
+def test_launch_count_per_layer_call():
+    """Kernels per moe_layer_forward: 8 for the bf16 decode layer (one-chunk permutation),
+    9 with the three-kernel permutation, + the FP8 scale preparation (act prep, 2 + 2
+    weight-scale conversions, scale gather), + the f32 family's bf16 conversions."""
+    assert bench.launches_per_step(inputs.SPECS["r1_decode"]) == 8
+    assert bench.launches_per_step(inputs.SPECS["r1_prefill"]) == 9
+    assert bench.launches_per_step(inputs.SPECS["kimi"]) == 9
+    assert bench.launches_per_step(inputs.SPECS["r1_prefill_fp8"]) == 15
+    assert bench.launches_per_step(inputs.SPECS["tiny"]) == 12
