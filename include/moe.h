@@ -39,7 +39,9 @@
  *    f32).  f32 inputs are rounded to bf16 (nearest even) on entry; the
  *    tensor cores compute in bf16 (or e4m3) with fp32 accumulation.  The
  *    router weights are bf16 for the bf16 and e4m3 families, f32 for f32.
- *    FP8 block scales must be powers of two.
+ *    FP8 block scales must be positive normal powers of two (exactly what the
+ *    tensor cores' UE8M0 scale factors represent); any other scale sets the
+ *    device status MOE_ERR_DEVICE_VALUE.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -65,7 +67,10 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,
   MOE_ERR_CUDA = 4,
   MOE_ERR_DEVICE_INDEX = 5,   /* device status: an expert index outside [0, E) */
-  MOE_ERR_TIMEOUT = 6         /* device status: a bounded in-kernel wait ran out */
+  MOE_ERR_TIMEOUT = 6,        /* device status: a bounded in-kernel wait ran out */
+  MOE_ERR_DEVICE_VALUE = 7    /* device status: an FP8 block scale that is not a positive,
+                                 normal power of two (the tensor cores take the scale's
+                                 exponent only); the results of that call are not valid */
 } moe_status;
 
 /* Router score function.

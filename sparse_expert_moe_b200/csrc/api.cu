@@ -443,13 +443,13 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
     uint4* wsf13 = at<uint4>(ws, L.wsf13);
     uint4* wsf2 = at<uint4>(ws, L.wsf2);
     st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(a), a_scale, n_rows,
-                                         static_cast<int>(d), nullptr, a_sf, stream));
+                                         static_cast<int>(d), nullptr, a_sf, status_word(ws), stream));
     if (st == MOE_OK)
       st = cuda_status(launch_weight_sf(w13_s, static_cast<size_t>(n_groups) * (2 * I / 128) * (d / 128),
-                                        wsf13, stream));
+                                        wsf13, status_word(ws), stream));
     if (st == MOE_OK)
       st = cuda_status(launch_weight_sf(w2_s, static_cast<size_t>(n_groups) * (d / 128) * (I / 128),
-                                        wsf2, stream));
+                                        wsf2, status_word(ws), stream));
     if (st == MOE_OK)
       st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, fp8_chunk_rows(n_rows),
                                    at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
@@ -550,13 +550,13 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   uint4* wsf2 = at<uint4>(ws, L.wsf2);
   if (fp8) {
     st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(x), x_scale, c.T,
-                                         static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf, s));
+                                         static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf, status, s));
     const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
     const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
-    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w13_s, E * n13, wsf13, s));
-    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w2_s, E * n2, wsf2, s));
-    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws13_s, S * n13, wsf13 + E * n13, s));
-    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws2_s, S * n2, wsf2 + E * n2, s));
+    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w13_s, E * n13, wsf13, status, s));
+    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w2_s, E * n2, wsf2, status, s));
+    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws13_s, S * n13, wsf13 + E * n13, status, s));
+    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws2_s, S * n2, wsf2 + E * n2, status, s));
     if (st != MOE_OK) return st;
     x_router = at<void>(ws, L.x_bf16);
   }
@@ -688,6 +688,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_DEVICE_INDEX: return "device: index or offset out of range";
     case MOE_ERR_TIMEOUT: return "device: bounded wait timed out";
+    case MOE_ERR_DEVICE_VALUE: return "device: FP8 block scale not a positive normal power of two";
   }
   return "unknown status";
 }

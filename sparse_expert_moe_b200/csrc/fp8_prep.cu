@@ -11,19 +11,25 @@
 #include <cuda_fp8.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
 
-// UE8M0 code of a power-of-two fp32 scale, replicated into the 4 bytes of a word.
-__device__ __forceinline__ uint32_t ue8m0x4(float s) {
-  return 0x01010101u * ((__float_as_uint(s) >> 23) & 0xFFu);
+// UE8M0 code of a power-of-two fp32 scale, replicated into the 4 bytes of a word.  A scale
+// that UE8M0 cannot hold exactly -- sign set, zero or subnormal, infinite or NaN, or any
+// mantissa bit set -- records MOE_ERR_DEVICE_VALUE in the status word.
+__device__ __forceinline__ uint32_t ue8m0x4(float s, int* status) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t e = (b >> 23) & 0xFFu;
+  if ((b & 0x807FFFFFu) != 0u || e == 0u || e == 0xFFu) record_status(status, kStatusDeviceValue);
+  return 0x01010101u * e;
 }
 
 // One thread per 16 activation bytes (16 e4m3 values, one 1x128 scale block).
 __global__ void act_prep_fp8_kernel(const uint4* __restrict__ x, const float* __restrict__ x_scale,
                                     int T, int d, uint4* __restrict__ x_bf16,
-                                    uint32_t* __restrict__ x_sf) {
+                                    uint32_t* __restrict__ x_sf, int* status) {
   const int vec_per_row = d / 16;
   const size_t n = static_cast<size_t>(T) * vec_per_row;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -46,14 +52,15 @@ __global__ void act_prep_fp8_kernel(const uint4* __restrict__ x, const float* __
       x_bf16[2 * i] = o[0];
       x_bf16[2 * i + 1] = o[1];
     }
-    if (x_sf && (v % 8) == 0) x_sf[static_cast<size_t>(kb) * T + t] = ue8m0x4(s);
+    if (x_sf && (v % 8) == 0) x_sf[static_cast<size_t>(kb) * T + t] = ue8m0x4(s, status);
   }
 }
 
-__global__ void weight_sf_kernel(const float* __restrict__ s, size_t n, uint4* __restrict__ out) {
+__global__ void weight_sf_kernel(const float* __restrict__ s, size_t n, uint4* __restrict__ out,
+                                 int* status) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint32_t w = ue8m0x4(s[i]);
+    const uint32_t w = ue8m0x4(s[i], status);
     out[i] = make_uint4(w, w, w, w);
   }
 }
@@ -81,17 +88,17 @@ unsigned grid_for(size_t n, int threads) {
 }  // namespace
 
 cudaError_t launch_act_prep_fp8(const uint8_t* x, const float* x_scale, int T, int d, void* x_bf16,
-                                uint32_t* x_sf, cudaStream_t s) {
+                                uint32_t* x_sf, int* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const size_t n = static_cast<size_t>(T) * (d / 16);
   act_prep_fp8_kernel<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), x_scale, T,
-                                                       d, static_cast<uint4*>(x_bf16), x_sf);
+                                                       d, static_cast<uint4*>(x_bf16), x_sf, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_weight_sf(const float* scales, size_t n, uint4* out, cudaStream_t s) {
+cudaError_t launch_weight_sf(const float* scales, size_t n, uint4* out, int* status, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  weight_sf_kernel<<<grid_for(n, 256), 256, 0, s>>>(scales, n, out);
+  weight_sf_kernel<<<grid_for(n, 256), 256, 0, s>>>(scales, n, out, status);
   return cudaGetLastError();
 }
 

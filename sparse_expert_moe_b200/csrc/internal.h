@@ -50,6 +50,7 @@ cudaError_t launch_route(const float* logits, int n_partials, long long partial_
 inline int router_splits(int64_t T, int64_t E, int64_t d) {
   const int64_t tiles = ((T + 127) / 128) * ((E + 127) / 128);
   const int64_t kb = d / 64;
+  if (tiles == 0) return 1;                 // empty batch: nothing to split
   int64_t s = tiles >= 48 ? 1 : 48 / tiles;
   if (s > 32) s = 32;
   if (s > kb) s = kb;
@@ -129,11 +130,12 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 
 // FP8 preparation kernels.
 // x e4m3 [T, d] + x_scale fp32 [T, d/128] -> x_bf16 [T, d] (exact) and x_sf [d/128][T]
-// (UE8M0 replicated x4).  Either output may be null.
+// (UE8M0 replicated x4).  Either output may be null.  Scales that are not positive normal
+// powers of two record MOE_ERR_DEVICE_VALUE in *status (both functions).
 cudaError_t launch_act_prep_fp8(const uint8_t* x, const float* x_scale, int T, int d, void* x_bf16,
-                                uint32_t* x_sf, cudaStream_t s);
+                                uint32_t* x_sf, int* status, cudaStream_t s);
 // fp32 power-of-two block scales [n] -> UE8M0 replicated x16 [n] (uint4).
-cudaError_t launch_weight_sf(const float* scales, size_t n, uint4* out, cudaStream_t s);
+cudaError_t launch_weight_sf(const float* scales, size_t n, uint4* out, int* status, cudaStream_t s);
 // x_perm_sf[kb][r] = x_sf[kb][perm_token[r]] for r < offsets_total (device).
 cudaError_t launch_gather_sf(const uint32_t* x_sf, int T, int kbs, const int32_t* perm_token,
                              const int32_t* total, int R, uint32_t* x_perm_sf, cudaStream_t s);

@@ -9,7 +9,7 @@
 namespace moe {
 
 // Status codes mirrored from include/moe.h for device code.
-enum : int { kStatusOk = 0, kStatusDeviceIndex = 5, kStatusTimeout = 6 };
+enum : int { kStatusOk = 0, kStatusDeviceIndex = 5, kStatusTimeout = 6, kStatusDeviceValue = 7 };
 
 // ~2 s at the B200's 1.965 GHz maximum SM clock: far beyond any legitimate wait
 // inside one kernel, short enough that a stuck kernel returns.

@@ -22,7 +22,8 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
-                4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_INDEX", 6: "MOE_ERR_TIMEOUT"}
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_INDEX", 6: "MOE_ERR_TIMEOUT",
+                7: "MOE_ERR_DEVICE_VALUE"}
 SCORE = {"softmax": 0, "sigmoid_bias": 1}
 DTYPE = {"f32": 0, "bf16": 1, "e4m3": 2}
 

@@ -30,6 +30,7 @@ def test_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     assert moe.moe_status_string(0) == "ok"
     assert "workspace" in moe.moe_status_string(3)
+    assert "power of two" in moe.moe_status_string(7)
     assert moe.moe_status_string(99) == "unknown status"
 
 
@@ -78,3 +79,16 @@ def test_workspace_too_small_rejected(lib):
     w = moe.MoeWeights(fake, 0, fake, fake, 0, 0, 0, 0, 0, 0)
     assert lib.moe_layer_forward(ctypes.byref(cfg), ctypes.byref(w), fake, None, fake, None, None,
                                  fake, 1024, None) == 3
+
+
+def test_empty_batch_is_a_no_op(lib):
+    """T = 0: the calls succeed without launching anything (no device needed here), and
+    the workspace of an empty batch has a size (its header)."""
+    cfg = moe.make_config(0, 256, 8, 2, 256, 1)
+    assert moe.moe_workspace_size(cfg) >= 256
+    fake = 256
+    w = moe.MoeWeights(fake, 0, fake, fake, 0, 0, fake, fake, 0, 0)
+    assert lib.moe_layer_forward(ctypes.byref(cfg), ctypes.byref(w), None, None, None, None, None,
+                                 fake, 1 << 20, None) == 0
+    assert lib.moe_route(ctypes.byref(cfg), None, None, None, None, None) == 0
+    assert lib.moe_combine(ctypes.byref(cfg), None, None, None, None, None, None) == 0

@@ -55,6 +55,33 @@ def test_grouped_ffn_vs_oracle(sizes, d, I):
     assert max_rel_err(got, ref) < TOL_BF16
 
 
+def test_grouped_ffn_all_groups_empty():
+    """Rows allocated but every group empty: the planner yields no tiles, the persistent
+    kernels exit at once, nothing is written and no status is set."""
+    d, I, G, n_rows = 256, 128, 5, 32
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0)
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    a = torch.randn((n_rows, d), device=DEV).to(torch.bfloat16)
+    w13 = torch.zeros((G, 2 * I, d), dtype=torch.bfloat16, device=DEV)
+    w2 = torch.zeros((G, d, I), dtype=torch.bfloat16, device=DEV)
+    y = torch.full((n_rows, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    offsets = torch.zeros(G + 1, dtype=torch.int32, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, offsets, n_rows, a, None, w13, None, w2, None, y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    assert bool((y == 7.0).all())
+
+
+def test_layer_empty_batch_leaves_output_untouched():
+    spec = inputs.custom_spec(8, 256, 8, 2, 128, 1)
+    wl = margin_workload(spec, seed=8)
+    layer = moe.DeviceLayer.from_workload(wl, DEV, T=0)
+    y = torch.full((1, 256), 3.0, dtype=torch.bfloat16, device=DEV)
+    moe.moe_layer_forward(layer.cfg, layer.weights, wl.x.to(DEV), None, y, None, None, layer.ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(layer.ws) == 0
+    assert bool((y == 3.0).all())
+
+
 def test_grouped_ffn_bad_offsets_set_device_status():
     d, I, G = 128, 128, 3
     cfg = moe.make_config(8, d, G, 1, I, 0)

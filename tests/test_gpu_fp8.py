@@ -106,6 +106,36 @@ def test_layer_fp8_custom(T, d, E, k, I, S):
     _check_fp8_layer(margin_workload(spec, seed=T + 1))
 
 
+@pytest.mark.parametrize("which,value", [("w13_s", 0.75), ("w2_s", 0.0), ("ws2_s", -0.5),
+                                         ("x_scale", 3.0), ("x_scale", float("inf"))])
+def test_layer_fp8_scale_outside_ue8m0_sets_device_status(which, value):
+    """A block scale the tensor cores' UE8M0 factors cannot hold exactly (not a positive
+    normal power of two) is reported through the device status, not silently rounded."""
+    spec = inputs.custom_spec(40, 256, 8, 2, 256, 1, act="e4m3", weight="e4m3")
+    wl = margin_workload(spec, seed=5)
+    layer = moe.DeviceLayer.from_workload(wl, DEV)
+    x, xs = wl.x.to(DEV), wl.x_scale.to(DEV).clone()
+    moe.moe_reset_device_status(layer.ws)
+    layer.forward(x, xs)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(layer.ws) == 0
+    if which == "x_scale":
+        xs[3, 1] = value
+        weights = layer.weights
+    else:
+        t = {k: v for k, v in layer.tensors.items()}
+        t[which] = t[which].clone()
+        t[which].view(-1)[-1] = value
+        weights = moe.make_weights(t["wr"], t["sel_bias"], t["w13"], t["w2"], t["ws13"], t["ws2"],
+                                   t["w13_s"], t["w2_s"], t["ws13_s"], t["ws2_s"])
+    y = layer.output(DEV)
+    moe.moe_layer_forward(layer.cfg, weights, x, xs, y, None, None, layer.ws)
+    assert moe.moe_read_device_status(layer.ws) == 7
+    moe.moe_reset_device_status(layer.ws)
+    layer.forward(x, wl.x_scale.to(DEV))
+    assert moe.moe_read_device_status(layer.ws) == 0
+
+
 @pytest.mark.slow
 def test_layer_fp8_full_size_sampled():
     wl = inputs.load_workload("r1_prefill_fp8")
