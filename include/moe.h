@@ -27,7 +27,8 @@
  *    MOE_ERR_WORKSPACE (workspace too small).  A launch error returns
  *    MOE_ERR_CUDA.
  *  - Faults the device detects (an expert index outside [0, E) fed to
- *    moe_permute; a bounded wait inside a kernel that ran out) are written to
+ *    moe_permute; an FP8 block scale that is not a positive normal power of
+ *    two; a bounded wait inside a kernel that ran out) are written to
  *    a status word in the first bytes of the workspace, never trapped; read
  *    it with moe_read_device_status.  The workspace must start zeroed once
  *    (moe_reset_device_status) before its first use.
