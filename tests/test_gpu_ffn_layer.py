@@ -29,6 +29,8 @@ def _bf16(a):
     ([300], 128, 384),                               # one group, three chunks, ragged tail
     ([1, 1, 1, 1], 512, 128),
     ([3, 0, 17, 32, 33], 1024, 256),                # decode-sized: 32-row chunks, 512-row weight tiles
+    # heavy groups over many 256-row chunks with ragged last chunks, then light groups
+    ([4000, 3000, 2600, 300, 5, 0, 70], 256, 2048),
 ])
 def test_grouped_ffn_vs_oracle(sizes, d, I):
     rng = np.random.default_rng(sum(sizes) + d + I)
