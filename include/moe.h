@@ -159,8 +159,15 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, c
  *    the call clears what must start at zero itself.  Calls whose kernels
  *    overlap on the GPU (several streams, or several host threads) race on it:
  *    serialise them.
- *  - No device status is recorded: pairs with an expert index outside [0, E)
- *    are dropped (inv_perm = -1, not counted in group_offsets). */
+ *  - Every dtype moe_permute takes: f32, bf16, and e4m3 rows, whose fp32
+ *    1x128 scales x_scale [T, d/128] are permuted into x_perm_scale
+ *    [T*k, d/128] (both required, non-NULL, when act is e4m3 and T > 0).
+ *  - No device status is recorded.  Pairs with an expert index outside [0, E)
+ *    are dropped (inv_perm = -1, not counted in group_offsets).  An expert
+ *    listed twice in one token's row is not detected: both slots get the same
+ *    permuted row, the group counts it once, and a combine over this result
+ *    adds that expert's output twice.  moe_permute reports both faults as
+ *    MOE_ERR_DEVICE_INDEX; call it where the indices are untrusted. */
 MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *topk_idx,
                                        const void *x, const float *x_scale, void *x_perm,
                                        float *x_perm_scale, int32_t *perm_token,
@@ -192,10 +199,14 @@ MOE_API moe_status moe_grouped_ffn(const moe_config *cfg, int32_t n_groups, cons
                            void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Weighted un-permute (the pseudocode's `out += weights[..., k] * e(x)` and
- * `out += s(x)`): out[t] = sum_j topk_w[t,j] * y_perm[inv_perm[t,j]] + y_shared[t],
- * summed in slot order in fp32 registers (no atomics), written as cfg->out.
+ * `out += s(x)`): out[t] = sum_j topk_w[t,j] * y_perm[inv_perm[t,j]]
+ * + sum_s y_shared[s, t], summed in slot order, then shared expert order, in
+ * fp32 registers (no atomics), rounded once and written as cfg->out.
  *   y_perm [T*k, d] bf16; inv_perm [T, k] int32 (entries outside [0, T*k) add 0);
- *   topk_w [T, k] fp32; y_shared [T, d] bf16 or NULL; y [T, d] (output). */
+ *   topk_w [T, k] fp32;
+ *   y_shared [cfg->n_shared, T, d] bf16: the shared experts' outputs stacked, or
+ *            NULL (nothing added; also when cfg->n_shared = 0 any pointer is ignored);
+ *   y [T, d] (output). */
 MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *inv_perm,
                        const float *topk_w, const void *y_shared, void *y, cudaStream_t stream);
 

@@ -50,8 +50,6 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                                           int32_t* inv_perm, int32_t* group_offsets,
                                           cudaStream_t stream) {
   using namespace moe;
-  (void)x_scale;
-  (void)x_perm_scale;
   moe_status st = validate_config(cfg);
   if (st != MOE_OK) return st;
   if (!group_offsets) return MOE_ERR_INVALID_ARG;
@@ -59,6 +57,9 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
     return MOE_ERR_INVALID_ARG;
+  // e4m3 rows come with one fp32 scale per 128 channels, permuted alongside the rows
+  const bool fp8 = cfg->act == MOE_E4M3;
+  if (fp8 && cfg->T > 0 && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
   const int64_t counts = static_cast<int64_t>(permute_chunks(cfg->T)) * cfg->E;
   if (counts > kMaxCountInts) return MOE_ERR_UNSUPPORTED;   // beyond the fixed scratch
   int32_t* scratch = scratch_on_current_device();
@@ -66,9 +67,11 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   // the scan ticket must start at zero; the array keeps whatever the last call left
   if (cudaMemsetAsync(scratch, 0, kHeaderInts * sizeof(int32_t), stream) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int elem = cfg->act == MOE_F32 ? 4 : 2;
+  // bytes per element of a row: f32 4, bf16 2, e4m3 1
+  const int elem = cfg->act == MOE_F32 ? 4 : (fp8 ? 1 : 2);
   const cudaError_t e = launch_permute(topk_idx, cfg->T, cfg->E, cfg->top_k, x, cfg->d_model * elem,
-                                       nullptr, 0, x_perm, nullptr, perm_token, inv_perm,
+                                       fp8 ? x_scale : nullptr, fp8 ? cfg->d_model / 128 : 0,
+                                       x_perm, fp8 ? x_perm_scale : nullptr, perm_token, inv_perm,
                                        group_offsets, scratch + kHeaderInts,
                                        reinterpret_cast<unsigned*>(scratch + 1), nullptr, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
