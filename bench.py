@@ -66,19 +66,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-FP8_PEAK_FILE = os.path.join(ROOT, "profiles", "fp8_peak.md")
+PEAKS_DATA = os.path.join(ROOT, "profiles", "peaks.json")
+
+
+def _peaks_data():
+    """Figures measured on this machine beyond MEASURED_PEAKS.json: the dense e4m3 GEMM peak
+    (``bench.py --fp8-peak``) and per-launch DRAM traffic from ncu captures."""
+    try:
+        with open(PEAKS_DATA) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
 
 
 def load_fp8_peak():
-    """Dense e4m3 GEMM throughput measured on this machine's B200s (``bench.py --fp8-peak``,
-    recorded in profiles/fp8_peak.md as ``fp8_tflops_sustained: X``), else None."""
-    try:
-        for line in open(FP8_PEAK_FILE):
-            if line.startswith("fp8_tflops_sustained:"):
-                return float(line.split(":", 1)[1])
-    except (OSError, ValueError):
-        pass
-    return None
+    """Sustained dense e4m3 GEMM throughput measured on this machine's B200s, else None."""
+    v = _peaks_data().get("fp8", {}).get("fp8_tflops_sustained")
+    return None if v is None else float(v)
 
 
 def measure_fp8_peak(dev, n=8192, seconds=4.0):
@@ -242,21 +246,17 @@ def bound_of(name):
 
 
 def read_traffic(kernel_key):
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the current
-    kernel source (else None)."""
+    """Per-launch DRAM bytes of an ncu capture, if it was taken on the current kernel
+    source (else None)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
-    try:
-        lines = open(path).read().splitlines()
-    except OSError:
+    ent = _peaks_data().get("traffic", {}).get(kernel_key)
+    if not ent:
         return None
     src = os.path.join(ROOT, "sparse_expert_moe_b200", "csrc", "grouped_gemm.cu")
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    for ln in lines:
-        parts = ln.split()
-        if len(parts) >= 3 and parts[0] == kernel_key and parts[2] == sha:
-            return float(parts[1])
-    return None
+    if ent.get("grouped_gemm_sha256_prefix") != sha:
+        return None
+    return float(ent["dram_bytes_per_launch"])
 
 
 # ---------------------------------------------------------------------------
@@ -589,7 +589,7 @@ def run_ours(args):
         if spec.weight == "e4m3":
             fp8 = load_fp8_peak()
             if fp8 is not None:
-                peak, peak_src = fp8, "measured e4m3 (profiles/fp8_peak.md)"
+                peak, peak_src = fp8, "measured e4m3 sustained (profiles/peaks.json)"
             else:
                 peak *= 2.0   # nominal fp8 : bf16 ratio of the dense tensor-core peaks
                 peak_src += " bf16 x 2 (nominal fp8 ratio)"

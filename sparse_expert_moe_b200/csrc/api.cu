@@ -478,7 +478,8 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
   if (!y_perm || !inv_perm || !topk_w || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(y) || !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
   const int R = cfg->T * cfg->top_k;
-  return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_shared, y_shared ? 1 : 0, cfg->T,
+  // y_shared holds the n_shared shared experts' outputs stacked [n_shared, T, d]
+  return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_shared, y_shared ? cfg->n_shared : 0, cfg->T,
                                     cfg->d_model, cfg->top_k, R, cfg->out == MOE_F32, y, stream));
 }
 

@@ -101,20 +101,22 @@ def test_grouped_ffn_bad_offsets_set_device_status():
 # combine alone
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("T,k,d,shared", [(1, 2, 128, False), (77, 8, 7168, True), (64, 16, 256, True)])
-def test_combine_vs_oracle(T, k, d, shared):
+@pytest.mark.parametrize("T,k,d,S", [(1, 2, 128, 0), (77, 8, 7168, 1), (64, 16, 256, 1),
+                                     (50, 4, 512, 3)])
+def test_combine_vs_oracle(T, k, d, S):
+    """S shared experts' outputs stacked [S, T, d] are all added."""
     rng = np.random.default_rng(T * k)
     R = T * k
     y_perm = _bf16(rng.standard_normal((R, d)))
     inv = rng.permutation(R).reshape(T, k).astype(np.int32)
     w = rng.uniform(0, 1, (T, k)).astype(np.float32)
-    ys = _bf16(rng.standard_normal((T, d))) if shared else None
-    cfg = moe.make_config(T, d, 16, k, 128, 1 if shared else 0)
+    ys = _bf16(rng.standard_normal((S, T, d))) if S else None
+    cfg = moe.make_config(T, d, 16, k, 128, S)
     y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
     moe.moe_combine(cfg, y_perm.to(DEV), torch.from_numpy(inv).to(DEV), torch.from_numpy(w).to(DEV),
                     None if ys is None else ys.to(DEV), y)
     ref = oracle.combine(y_perm.double().numpy(), inv, w.astype(np.float64),
-                         None if ys is None else [ys.double().numpy()])
+                         None if ys is None else list(ys.double().numpy()))
     got = y.float().cpu().numpy()
     # one bf16 rounding of an fp32 sum
     assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5 * np.abs(ref).max())
