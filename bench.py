@@ -194,7 +194,8 @@ def work_model(spec, offsets):
     the routed and shared rows plus the router's 2 * T * d * E.
     """
     T, d, E, k, I, S = spec.T, spec.d_model, spec.E, spec.top_k, spec.d_ff, spec.n_shared
-    wb = 1 if spec.weight == "e4m3" else 2
+    # weight bytes per element: MXFP4 = half a byte + one E8M0 byte per 32 elements
+    wb = {"e4m3": 1.0, "e2m1": 0.5 + 1.0 / 32}.get(spec.weight, 2.0)
     ab = 1 if spec.act == "e4m3" else 2
     sizes = np.diff(offsets)
     touched = int((sizes > 0).sum())
@@ -316,6 +317,8 @@ def _weight_values(w, s):
     import torch
     if s is None:
         return w.double().numpy()
+    if s.dtype == torch.uint8:           # MXFP4: packed E2M1 codes + E8M0 scale codes
+        return oracle.dequantize_mxfp4(w.numpy(), s.numpy())
     return oracle.dequantize_blocks(w.view(torch.uint8).numpy(), s.numpy(), 128, 128)
 
 
@@ -473,6 +476,64 @@ def time_e2e(layer, wl, y, idx, gw, stream, K, dev, barrier, max_over_ranks):
     return ms, h2d, d2h
 
 
+def time_staged(moe, layer, weights, x, xs, y, idx, gw, K, stream, dev, barrier, max_over_ranks):
+    """K ``moe_layer_forward_staged`` calls between a barrier + synchronize on both sides:
+    (max over ranks of the total ms, mean ms per stage from the in-place events)."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)   # create the events before they are handed to the library
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(K):
+        moe.moe_layer_forward_staged(layer.cfg, weights, x, xs, y, idx, gw, layer.ws, evs[i], stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = max_over_ranks(start.elapsed_time(end))
+    stage_ms = {s: 0.0 for s in moe.STAGES}
+    for row in evs:
+        for j, s in enumerate(moe.STAGES):
+            stage_ms[s] += row[j].elapsed_time(row[j + 1]) / K
+    return ms_total, stage_ms
+
+
+def decode_uniform(moe, inputs, layer, wl, y, idx, gw, K, W, stream, dev, barrier, max_over_ranks,
+                   peaks):
+    """The uniformly routed R1 decode batch (no selection bias: about 252 of 256 experts
+    touched, the full weight traffic of a decode step) on the same resident weights, timed
+    like the main line; reported beside it."""
+    import torch
+    wu = inputs.load_workload("r1_decode_uniform", reuse=wl)
+    xu = wu.x.to(dev)
+    t = layer.tensors
+    weights = moe.make_weights(t["wr"], None, t["w13"], t["w2"], t["ws13"], t["ws2"])
+    for _ in range(W):
+        moe.moe_layer_forward(layer.cfg, weights, xu, None, y, idx, gw, layer.ws, stream)
+    torch.cuda.synchronize(dev)
+    ms_total, stage_ms = time_staged(moe, layer, weights, xu, None, y, idx, gw, K, stream, dev,
+                                     barrier, max_over_ranks)
+    ms = ms_total / K
+    spec = wu.spec
+    sizes = np.bincount(idx.cpu().numpy().ravel(), minlength=spec.E)
+    wm = work_model(spec, np.concatenate([[0], np.cumsum(sizes)]))
+    hbm = peaks["hbm_gbs"]
+    gbs = lambda b, t: b / (t * 1e-3) / 1e9
+    return {"workload": "r1_decode_uniform", "ms_per_step": ms, "value": spec.T / (ms * 1e-3),
+            "unit": "tokens/s", "touched_experts": wm["touched"],
+            "weight_bytes_touched": wm["layer_weight_bytes"],
+            "hbm_frac_layer": gbs(wm["layer_weight_bytes"], ms) / hbm,
+            "ffn1": {"ms": stage_ms["ffn1"], "gbs": gbs(wm["ffn1_bytes"], stage_ms["ffn1"]),
+                     "frac": gbs(wm["ffn1_bytes"], stage_ms["ffn1"]) / hbm},
+            "ffn2": {"ms": stage_ms["ffn2"], "gbs": gbs(wm["ffn2_bytes"], stage_ms["ffn2"]),
+                     "frac": gbs(wm["ffn2_bytes"], stage_ms["ffn2"]) / hbm},
+            "stages_ms": stage_ms}
+
+
 def launches_per_step(spec):
     """Kernels one ``moe_layer_forward`` launches: router GEMM, route, permute (count and
     gather for T <= 256, else count, rank and gather), plan, FFN1, FFN2, combine; the
@@ -482,7 +543,9 @@ def launches_per_step(spec):
     if spec.act == "f32":
         n += 4 + (2 if spec.n_shared else 0)
     if spec.act == "e4m3":
-        n += 1 + 2 + (2 if spec.n_shared else 0) + 1
+        n += 1 + 1                     # activation scale preparation, permuted-row scales
+    if spec.weight == "e4m3":
+        n += 2 + (2 if spec.n_shared else 0)   # weight block scales -> UE8M0
     return n
 
 
@@ -537,43 +600,29 @@ def run_ours(args):
 
     # timed steps: stage events recorded in place
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
-    for row in evs:
-        for e in row:
-            e.record(stream)   # create the events before they are handed to the library
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
-    barrier()
-    torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
-        start.record(stream)
-        for i in range(K):
-            moe.moe_layer_forward_staged(layer.cfg, layer.weights, x, xs, y, idx, gw, layer.ws, evs[i],
-                                         stream)
-        end.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier()
-    ms_total = max_over_ranks(start.elapsed_time(end))
+        ms_total, stage_ms = time_staged(moe, layer, layer.weights, x, xs, y, idx, gw, K, stream,
+                                         dev, barrier, max_over_ranks)
     ms_step = ms_total / K
-    stage_ms = {s: 0.0 for s in moe.STAGES}
-    for row in evs:
-        for j, s in enumerate(moe.STAGES):
-            stage_ms[s] += row[j].elapsed_time(row[j + 1]) / K
     status = moe.moe_read_device_status(layer.ws)
 
     # end to end through the public call, pipelined as a serving loop runs it
     e2e_ms, h2d, d2h = time_e2e(layer, wl, y, idx, gw, stream, K, dev, barrier, max_over_ranks)
+    idx_np = idx.cpu().numpy()
+    peaks, peak_src = load_peaks()
+    uniform = None
+    if name == "r1_decode" and not args.experts:
+        uniform = decode_uniform(moe, inputs, layer, wl, y, idx, gw, K, args.warmup, stream, dev,
+                                 barrier, max_over_ranks, peaks)
 
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
 
-    idx_np = idx.cpu().numpy()
     sizes = np.bincount(idx_np.ravel(), minlength=spec.E)
     off = np.concatenate([[0], np.cumsum(sizes)])
     wm = work_model(spec, off)
-    peaks, peak_src = load_peaks()
     bound = bound_of(name)
     if bound == "hbm":
         dom = "ffn1"
@@ -605,7 +654,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if spec.weight == "e4m3" else "bf16", "data": "synthetic",
+        "dtype": {"e4m3": "e4m3", "e2m1": "e2m1 x e4m3"}.get(spec.weight, "bf16"),
+        "data": "synthetic",
         "config": {"workload": name if not args.experts else
                    f"{name} with E={spec.E}, T={spec.T} (profiling case)",
                    "T": spec.T, "d_model": spec.d_model, "E": spec.E,
@@ -613,7 +663,8 @@ def run_ours(args):
                    "score": spec.score, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: each step streams "
                          f"{wm['layer_weight_bytes'] / 1e9:.1f} GB of expert weights"},
-        "roofline": {"bound": bound, "kernel": f"{dom} (grouped_gemm_kernel<1>)",
+        "roofline": {"bound": bound,
+                     "kernel": f"{dom} (grouped_gemm_kernel<{ {'e4m3': 3, 'e2m1': 7}.get(spec.weight, 1)}>)",
                      "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": unit,
                      "frac": achieved / peak, "traffic": read_traffic(f"ffn1_{name}"),
                      "units": units_note},
@@ -635,6 +686,8 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "device_status": status,
     }
+    if uniform is not None:
+        line["decode_uniform"] = uniform
     if not args.no_cpu_baseline and world == 1:
         host = {n: getattr(wl, n) for n in ("w13", "w2", "ws13", "ws2", "w13_s", "w2_s", "ws13_s",
                                             "ws2_s")}

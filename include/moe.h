@@ -37,12 +37,14 @@
  *  - dtypes: activations MOE_BF16, MOE_E4M3 (with fp32 1x128 scales) or
  *    MOE_F32; weights the same family (bf16 weights with bf16 activations,
  *    e4m3 weights + fp32 128x128 block scales with e4m3 activations, f32 with
- *    f32).  f32 inputs are rounded to bf16 (nearest even) on entry; the
- *    tensor cores compute in bf16 (or e4m3) with fp32 accumulation.  The
- *    router weights are bf16 for the bf16 and e4m3 families, f32 for f32.
+ *    f32), or MOE_E2M1 (MXFP4) weights with MOE_E4M3 activations.  f32 inputs
+ *    are rounded to bf16 (nearest even) on entry; the tensor cores compute in
+ *    bf16 (or e4m3 / e2m1 x e4m3) with fp32 accumulation.  The router weights
+ *    are bf16 for the bf16, e4m3 and e2m1 families, f32 for f32.
  *    FP8 block scales must be positive normal powers of two (exactly what the
  *    tensor cores' UE8M0 scale factors represent); any other scale sets the
- *    device status MOE_ERR_DEVICE_VALUE.
+ *    device status MOE_ERR_DEVICE_VALUE.  MXFP4 scale bytes are used as given
+ *    (code 0xFF, NaN in E8M0, gives undefined results).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -86,7 +88,10 @@ typedef enum {
  * equal keys by lower expert index. */
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_BIAS = 1 } moe_score_fn;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
+/* MOE_E2M1: FP4 weights in the OCP MXFP4 format -- E2M1 codes packed two per byte (element
+ * 2j in the low nibble of byte j), one E8M0 scale byte (2^(code - 127)) per 32 consecutive
+ * elements along K -- taken with e4m3 activations ("FP8/FP4 grouped GEMM", GC-MoE title). */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2, MOE_E2M1 = 3 } moe_dtype;
 
 /* The layer's sizes: T tokens x d_model activations, E routed experts, top_k,
  * expert intermediate size d_ff (I), n_shared always-on shared experts of
@@ -102,15 +107,19 @@ typedef struct {
  *   sel_bias [E] fp32      selection bias (SIGMOID_BIAS only; may be NULL = 0)
  *   w13    [E, 2I, d]      per expert: W1 (gate, rows 0..I-1) over W3 (up, rows I..2I-1)
  *   w2     [E, d, I]       per expert down projection
- *   w13_s  [E, 2I/128, d/128] fp32, w2_s [E, d/128, I/128] fp32: e4m3 block scales
+ *   w13_s, w2_s            block scales of the weights:
+ *                          e4m3: fp32 [E, 2I/128, d/128] and [E, d/128, I/128];
+ *                          e2m1: uint8 E8M0 codes [E, 2I, d/32] and [E, d, I/32]
+ *                          (w13 is then [E, 2I, d/2] bytes, w2 [E, d, I/2]; both
+ *                          32-byte aligned); unused (NULL) otherwise
  *   ws13 [S, 2I, d], ws2 [S, d, I] (+ ws13_s, ws2_s): shared experts (NULL when S = 0) */
 typedef struct {
   const void *wr;
   const float *sel_bias;
   const void *w13, *w2;
-  const float *w13_s, *w2_s;
+  const void *w13_s, *w2_s;
   const void *ws13, *ws2;
-  const float *ws13_s, *ws2_s;
+  const void *ws13_s, *ws2_s;
 } moe_weights;
 
 /* Bytes of workspace moe_layer_forward / moe_permute / moe_grouped_ffn need
@@ -188,14 +197,15 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *top
  *   a               [offsets[G], d] rows (cfg->act); a_scale [rows, d/128] fp32
  *                   for e4m3, else NULL.  For the f32 family a, w13 and w2 are
  *                   rounded to bf16 into the workspace first.
- *   w13, w2         [G, 2I, d], [G, d, I] (+ block scales for e4m3)
+ *   w13, w2         [G, 2I, d], [G, d, I] (+ block scales for e4m3 and e2m1 weights,
+ *                   laid out as in moe_weights)
  *   y               [offsets[G], d] bf16 output
  * The shared expert is this call with n_groups = 1, offsets {0, T}, a = x.
  * The intermediate h lives in the workspace.  A persistent tcgen05/TMA kernel
  * walks the groups with a device-side tile scheduler (no host sync). */
 MOE_API moe_status moe_grouped_ffn(const moe_config *cfg, int32_t n_groups, const int32_t *group_offsets,
                            int32_t n_rows, const void *a, const float *a_scale, const void *w13,
-                           const float *w13_s, const void *w2, const float *w2_s, void *y,
+                           const void *w13_s, const void *w2, const void *w2_s, void *y,
                            void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Weighted un-permute (the pseudocode's `out += weights[..., k] * e(x)` and

@@ -39,6 +39,11 @@ single steps.  Readings of points the pages leave open:
 * FP8 inputs are e4m3 codes times power-of-two block scales; the oracle
   decodes the codes from the OCP OFP8 E4M3 definition and multiplies the scale
   in, exactly, in fp64.
+* FP4 ("FP8/FP4 Grouped GEMM" in the GC-MoE title names the precision, not the
+  format).  Reading: the OCP Microscaling (MX) MXFP4 format -- E2M1 elements,
+  two per byte (the even element in the low nibble), one E8M0 scale per 32
+  consecutive elements along K.  The oracle decodes both from their
+  definitions and multiplies, exactly, in fp64.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` (closed forms,
 brute force over expert subsets, library special cases, invariants and the
@@ -86,6 +91,47 @@ def dequantize_blocks(q_codes, scales, block_rows: int, block_cols: int) -> np.n
     s = np.asarray(scales, dtype=np.float64)
     s = np.repeat(np.repeat(s, block_rows, axis=0), block_cols, axis=1)
     return v * s[: v.shape[0], : v.shape[1]]
+
+
+def decode_e2m1(codes) -> np.ndarray:
+    """Decode 4-bit FP4 E2M1 codes (the low 4 bits of each value) to fp64.
+
+    Format (OCP Microscaling Formats (MX) v1.0, element type FP4 E2M1): 1 sign
+    bit, 2 exponent bits with bias 1, 1 mantissa bit; exponent field 0 encodes
+    the subnormals m/2 * 2^0; no infinities or NaN, so the largest magnitude is
+    1.5 * 2^2 = 6.
+    """
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    exp = (c >> 1) & 0x3
+    man = (c & 0x1).astype(np.float64)
+    normal = (1.0 + man / 2.0) * np.exp2(exp.astype(np.float64) - 1.0)
+    sub = man / 2.0
+    return sign * np.where(exp == 0, sub, normal)
+
+
+def unpack_fp4(packed) -> np.ndarray:
+    """[R, C/2] bytes of packed FP4 codes -> [R, C] codes: byte j holds element 2j in its
+    low nibble and element 2j+1 in its high nibble."""
+    b = np.asarray(packed, np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def decode_e8m0(codes) -> np.ndarray:
+    """Decode E8M0 scale codes to fp64 (OCP MX v1.0, scale type E8M0): 8 exponent bits,
+    bias 127, no sign and no mantissa, value 2^(code - 127); code 0xFF is NaN."""
+    c = np.asarray(codes, np.uint8).astype(np.float64)
+    return np.where(c == 255.0, np.nan, np.exp2(c - 127.0))
+
+
+def dequantize_mxfp4(packed, scale_codes, block: int = 32) -> np.ndarray:
+    """MXFP4 to fp64: value[r, c] = e2m1(code[r, c]) * e8m0(scale[r, c // block])."""
+    v = decode_e2m1(unpack_fp4(packed))
+    s = decode_e8m0(scale_codes)
+    return v * np.repeat(s, block, axis=-1)[..., : v.shape[-1]]
 
 
 # ---------------------------------------------------------------------------

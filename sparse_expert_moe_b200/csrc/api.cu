@@ -36,7 +36,8 @@ struct Layout {
     rows_all = R + S * T;
     n_chunk_max = max_chunks(rows_all, E + S);
     const bool f32 = c.act == MOE_F32;
-    const bool fp8 = c.act == MOE_E4M3;
+    const bool fp8 = c.act == MOE_E4M3;            // e4m3 activations (e4m3 or FP4 weights)
+    const bool w8 = c.weight == MOE_E4M3;          // fp32 block scales re-encoded per call
     size_t o = kHeaderBytes;
     auto take = [&](size_t bytes) {
       const size_t at = o;
@@ -65,8 +66,8 @@ struct Layout {
     x_perm_sf = take(fp8 ? 4 * (d / 128) * R : 0);
     h_sf = take(fp8 ? 4 * (I / 128) * rows_all : 0);
     a_sf = take(fp8 ? 4 * (d / 128) * rows_all : 0);
-    wsf13 = take(fp8 ? 16 * (E + S) * (2 * I / 128) * (d / 128) : 0);
-    wsf2 = take(fp8 ? 16 * (E + S) * (d / 128) * (I / 128) : 0);
+    wsf13 = take(w8 ? 16 * (E + S) * (2 * I / 128) * (d / 128) : 0);
+    wsf2 = take(w8 ? 16 * (E + S) * (d / 128) * (I / 128) : 0);
     total = o;
   }
 };
@@ -78,6 +79,11 @@ inline T* at(void* ws, size_t off) {
 inline int* status_word(void* ws) { return at<int>(ws, kHdrStatus * sizeof(int)); }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+// bytes of a weight row of `k` elements
+inline int64_t weight_row_bytes(const moe_config& c, int64_t k) {
+  return c.weight == MOE_E2M1 ? k / 2 : (c.weight == MOE_E4M3 ? k : (c.weight == MOE_F32 ? 4 * k : 2 * k));
+}
 
 moe_status check_config(const moe_config* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -94,7 +100,8 @@ moe_status check_config(const moe_config* c) {
   const bool fam_bf16 = c->act == MOE_BF16 && c->weight == MOE_BF16;
   const bool fam_f32 = c->act == MOE_F32 && c->weight == MOE_F32;
   const bool fam_fp8 = c->act == MOE_E4M3 && c->weight == MOE_E4M3;
-  if (!(fam_bf16 || fam_f32 || fam_fp8)) return MOE_ERR_UNSUPPORTED;
+  const bool fam_w4a8 = c->act == MOE_E4M3 && c->weight == MOE_E2M1;
+  if (!(fam_bf16 || fam_f32 || fam_fp8 || fam_w4a8)) return MOE_ERR_UNSUPPORTED;
   if (c->out != MOE_BF16 && c->out != MOE_F32) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -107,9 +114,11 @@ int bf16_chunk_rows(int64_t max_group) {
   return max_group <= kChunkRows ? kChunkRowsNarrow : kChunkRowsWide;
 }
 
-// FP8 chunk rows: 112, or 224 once groups can exceed 112 rows (FFN2 tiles of 224
-// tokens, FFN1 tiles of half a chunk).
+// FP8 / FP4-weight chunk rows: 32 for decode-sized batches (groups of at most 128 rows:
+// small token tiles leave shared memory to the weight stream), else 112, or 224 once
+// groups can exceed 112 rows (FFN2 tiles of 224 tokens, FFN1 tiles of half a chunk).
 int fp8_chunk_rows(int64_t max_group) {
+  if (max_group <= kChunkRows) return kChunkRowsNarrow;
   return max_group <= kChunkRowsFP8 ? kChunkRowsFP8 : 2 * kChunkRowsFP8;
 }
 
@@ -155,6 +164,19 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_fp4(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols == 0 || cols % 128) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols / 2};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                   uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -183,20 +205,39 @@ void copy_maps(CUtensorMap (&dst)[4], const CUtensorMap (&src)[4]) {
   for (int i = 0; i < 4; ++i) dst[i] = src[i];
 }
 
+// One segment of the FP8 block-scaled expert GEMMs: token rows `a` (e4m3) with their
+// UE8M0 scale factors a_sf [d/128][a_rows], and `groups` experts' weights -- e4m3 with
+// UE8M0 block scale factors wsf13 / wsf2 (re-encoded from the caller's fp32 128x128
+// scales), or FP4 (packed E2M1) with the caller's E8M0 codes wsc13 [rows][d/32] /
+// wsc2 [rows][I/32].
+struct Fp8Seg {
+  const void* a;
+  const uint32_t* a_sf;
+  int64_t a_rows;
+  const void* w13;
+  const void* w2;
+  const uint4* wsf13;
+  const uint4* wsf2;
+  const uint8_t* wsc13;
+  const uint8_t* wsc2;
+  int64_t groups;
+};
+
+bool weight_map(CUtensorMap* m, const void* w, int64_t rows, int64_t cols, bool w4) {
+  return w4 ? make_tmap_fp4(m, w, rows, cols, 128) : make_tmap_u8(m, w, rows, cols, 128);
+}
+
 // The FP8 block-scaled expert GEMMs over a chunk list already planned into the
-// workspace.  seg 0: routed rows a0 (token scales a0_sf [d/128][a0_rows]) with
-// weights w13_0 / w2_0 and their UE8M0 block scales wsf13_0 / wsf2_0 (G0 groups);
-// seg 1: shared experts on rows a1 (scales a1_sf) or absent (S = 0).  h (e4m3) and
-// its scales live in the workspace; y has rows_all rows.
-moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const void* a0,
-                       const uint32_t* a0_sf, int64_t a0_rows, const void* w13_0, const void* w2_0,
-                       const uint4* wsf13_0, const uint4* wsf2_0, int64_t G0, const void* a1,
-                       const uint32_t* a1_sf, int64_t a1_rows, const void* w13_1, const void* w2_1,
-                       const uint4* wsf13_1, const uint4* wsf2_1, int64_t S, int64_t rows_all,
-                       void* y, int chunk_rows, cudaStream_t s, cudaEvent_t* ev = nullptr) {
+// workspace: seg0 the routed rows, seg1 the shared experts (groups = 0: absent).  h
+// (e4m3) and its scales live in the workspace; y has rows_all rows.
+moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8Seg& s0,
+                       const Fp8Seg& s1, int64_t rows_all, void* y, int chunk_rows, cudaStream_t s,
+                       cudaEvent_t* ev = nullptr) {
   const int64_t d = c.d_model, I = c.d_ff;
+  const bool w4 = c.weight == MOE_E2M1;
   void* h = at<void>(ws, L.h);
   uint32_t* h_sf = at<uint32_t>(ws, L.h_sf);
+  const Fp8Seg* seg[2] = {&s0, s1.groups > 0 ? &s1 : &s0};
   GemmLaunch g{};
   g.chunks = at<Chunk>(ws, L.chunks);
   g.n_chunks = at<int32_t>(ws, kHdrNChunks * sizeof(int));
@@ -205,31 +246,23 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
   g.status = status_word(ws);
   g.num_sms = num_sms();
 
-  // FFN1 tiles hold 112 tokens (half a 224-row chunk when chunks are 224 rows); FFN2
-  // tiles are one chunk wide
-  g.mode = kFFN1F8;
+  // FFN1 tiles hold 32 tokens on decode-sized chunks, else 112 (half a 224-row chunk when
+  // chunks are 224 rows); FFN2 tiles are one chunk wide
+  g.mode = w4 ? kFFN1F4 : kFFN1F8;
   g.halves = chunk_rows == 2 * kChunkRowsFP8;
-  if (!make_tmap_u8(&g.wmap[0], w13_0, G0 * 2 * I, d, 128) || !make_tok_maps(g.tmap[0], a0, a0_rows, d, true))
-    return MOE_ERR_CUDA;
-  g.wsf[0] = wsf13_0;
-  g.tsf[0] = a0_sf;
-  g.tsf_ld[0] = static_cast<int>(a0_rows);
-  g.tsf_rows[0] = static_cast<int>(a0_rows);
-  if (S > 0) {
-    if (!make_tmap_u8(&g.wmap[1], w13_1, S * 2 * I, d, 128) || !make_tok_maps(g.tmap[1], a1, a1_rows, d, true))
+  g.tile_tokens = chunk_rows == kChunkRowsNarrow ? kChunkRowsNarrow : kChunkRows;
+  for (int i = 0; i < 2; ++i) {
+    const Fp8Seg& q = *seg[i];
+    if (!weight_map(&g.wmap[i], q.w13, q.groups * 2 * I, d, w4) ||
+        !make_tok_maps(g.tmap[i], q.a, q.a_rows, d, true))
       return MOE_ERR_CUDA;
-    g.wsf[1] = wsf13_1;
-    g.tsf[1] = a1_sf;
-    g.tsf_ld[1] = static_cast<int>(a1_rows);
-    g.tsf_rows[1] = static_cast<int>(a1_rows);
-  } else {
-    g.wmap[1] = g.wmap[0];
-    copy_maps(g.tmap[1], g.tmap[0]);
-    g.wsf[1] = g.wsf[0];
-    g.tsf[1] = g.tsf[0];
-    g.tsf_ld[1] = g.tsf_ld[0];
-    g.tsf_rows[1] = g.tsf_rows[0];
+    g.wsf[i] = q.wsf13;
+    g.wsc[i] = q.wsc13;
+    g.tsf[i] = q.a_sf;
+    g.tsf_ld[i] = static_cast<int>(q.a_rows);
+    g.tsf_rows[i] = static_cast<int>(q.a_rows);
   }
+  g.wsc_ld = static_cast<int>(d / 32);
   g.n_mblk = static_cast<int>(I / 128);
   g.k_blocks = static_cast<int>(d / 128);
   g.w_rows_per_group = static_cast<int>(2 * I);
@@ -244,25 +277,21 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const voi
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
-  g.mode = kFFN2F8;
+  g.mode = w4 ? kFFN2F4 : kFFN2F8;
   g.halves = false;
   g.tile_tokens = chunk_rows;
-  if (!make_tmap_u8(&g.wmap[0], w2_0, G0 * d, I, 128) || !make_tok_maps(g.tmap[0], h, rows_all, I, true))
-    return MOE_ERR_CUDA;
-  g.wsf[0] = wsf2_0;
-  if (S > 0) {
-    if (!make_tmap_u8(&g.wmap[1], w2_1, S * d, I, 128)) return MOE_ERR_CUDA;
-    g.wsf[1] = wsf2_1;
-  } else {
-    g.wmap[1] = g.wmap[0];
-    g.wsf[1] = g.wsf[0];
-  }
+  if (!make_tok_maps(g.tmap[0], h, rows_all, I, true)) return MOE_ERR_CUDA;
   copy_maps(g.tmap[1], g.tmap[0]);
   for (int i = 0; i < 2; ++i) {
+    const Fp8Seg& q = *seg[i];
+    if (!weight_map(&g.wmap[i], q.w2, q.groups * d, I, w4)) return MOE_ERR_CUDA;
+    g.wsf[i] = q.wsf2;
+    g.wsc[i] = q.wsc2;
     g.tsf[i] = h_sf;
     g.tsf_ld[i] = static_cast<int>(rows_all);
     g.tsf_rows[i] = static_cast<int>(rows_all);
   }
+  g.wsc_ld = static_cast<int>(I / 32);
   g.n_mblk = static_cast<int>(d / 128);
   g.k_blocks = static_cast<int>(I / 128);
   g.w_rows_per_group = static_cast<int>(d);
@@ -403,16 +432,15 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
 
 moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_t* group_offsets,
                            int32_t n_rows, const void* a, const float* a_scale, const void* w13,
-                           const float* w13_s, const void* w2, const float* w2_s, void* y,
+                           const void* w13_s, const void* w2, const void* w2_s, void* y,
                            void* ws, size_t ws_bytes, cudaStream_t stream) {
-  (void)a_scale;
-  (void)w13_s;
-  (void)w2_s;
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (n_groups <= 0 || n_groups > 1024 || n_rows < 0) return MOE_ERR_INVALID_ARG;
   if (!group_offsets || !a || !w13 || !w2 || !y || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(w13) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  // packed FP4 weights are loaded by TMA from 32-byte aligned bases
+  if (cfg->weight == MOE_E2M1 && (!aligned32(w13) || !aligned32(w2))) return MOE_ERR_INVALID_ARG;
   const Layout L(*cfg);
   if (n_rows > L.rows_all) return MOE_ERR_UNSUPPORTED;
   // the workspace's chunk list and group tables are sized for E + n_shared groups
@@ -439,26 +467,35 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
   }
   if (cfg->act == MOE_E4M3) {
     if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
+    const bool w4 = cfg->weight == MOE_E2M1;
     uint32_t* a_sf = at<uint32_t>(ws, L.a_sf);
-    uint4* wsf13 = at<uint4>(ws, L.wsf13);
-    uint4* wsf2 = at<uint4>(ws, L.wsf2);
+    Fp8Seg s0{a, a_sf, n_rows, w13, w2, nullptr, nullptr, nullptr, nullptr, n_groups};
     st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(a), a_scale, n_rows,
                                          static_cast<int>(d), nullptr, a_sf, status_word(ws), stream));
+    if (w4) {
+      s0.wsc13 = static_cast<const uint8_t*>(w13_s);
+      s0.wsc2 = static_cast<const uint8_t*>(w2_s);
+    } else {
+      s0.wsf13 = at<uint4>(ws, L.wsf13);
+      s0.wsf2 = at<uint4>(ws, L.wsf2);
+      if (st == MOE_OK)
+        st = cuda_status(launch_weight_sf(static_cast<const float*>(w13_s),
+                                          static_cast<size_t>(n_groups) * (2 * I / 128) * (d / 128),
+                                          at<uint4>(ws, L.wsf13), status_word(ws), stream));
+      if (st == MOE_OK)
+        st = cuda_status(launch_weight_sf(static_cast<const float*>(w2_s),
+                                          static_cast<size_t>(n_groups) * (d / 128) * (I / 128),
+                                          at<uint4>(ws, L.wsf2), status_word(ws), stream));
+    }
+    const int chunk_rows = fp8_chunk_rows(n_rows);
     if (st == MOE_OK)
-      st = cuda_status(launch_weight_sf(w13_s, static_cast<size_t>(n_groups) * (2 * I / 128) * (d / 128),
-                                        wsf13, status_word(ws), stream));
-    if (st == MOE_OK)
-      st = cuda_status(launch_weight_sf(w2_s, static_cast<size_t>(n_groups) * (d / 128) * (I / 128),
-                                        wsf2, status_word(ws), stream));
-    if (st == MOE_OK)
-      st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, fp8_chunk_rows(n_rows),
+      st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, chunk_rows,
                                    at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
-                               at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
+                                   at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
                                    status_word(ws), stream));
     if (st != MOE_OK) return st;
-    return run_ffn_fp8(*cfg, L, ws, a, a_sf, n_rows, w13, w2, wsf13, wsf2, n_groups, nullptr,
-                       nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0, n_rows, y,
-                       fp8_chunk_rows(n_rows), stream);
+    const Fp8Seg none{};
+    return run_ffn_fp8(*cfg, L, ws, s0, none, n_rows, y, chunk_rows, stream);
   }
   const int chunk_rows = bf16_chunk_rows(n_rows);
   st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, chunk_rows,
@@ -506,8 +543,13 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
       !aligned16(wts->w2) || !aligned16(wts->ws13) || !aligned16(wts->ws2))
     return MOE_ERR_INVALID_ARG;
   const bool fp8 = c.act == MOE_E4M3;
+  const bool w4 = c.weight == MOE_E2M1;
   if (fp8 && (!x_scale || !wts->w13_s || !wts->w2_s ||
               (c.n_shared > 0 && (!wts->ws13_s || !wts->ws2_s))))
+    return MOE_ERR_INVALID_ARG;
+  // packed FP4 weights are loaded by TMA from 32-byte aligned bases
+  if (w4 && (!aligned32(wts->w13) || !aligned32(wts->w2) || !aligned32(wts->ws13) ||
+             !aligned32(wts->ws2)))
     return MOE_ERR_INVALID_ARG;
   const Layout L(c);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -549,15 +591,20 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   uint32_t* x_sf = at<uint32_t>(ws, L.x_sf);
   uint4* wsf13 = at<uint4>(ws, L.wsf13);
   uint4* wsf2 = at<uint4>(ws, L.wsf2);
+  const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
+  const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
   if (fp8) {
     st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(x), x_scale, c.T,
                                          static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf, status, s));
-    const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
-    const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
-    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w13_s, E * n13, wsf13, status, s));
-    if (st == MOE_OK) st = cuda_status(launch_weight_sf(wts->w2_s, E * n2, wsf2, status, s));
-    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws13_s, S * n13, wsf13 + E * n13, status, s));
-    if (st == MOE_OK && S > 0) st = cuda_status(launch_weight_sf(wts->ws2_s, S * n2, wsf2 + E * n2, status, s));
+    if (!w4) {   // e4m3 weights: fp32 block scales -> UE8M0 scale factors
+      auto wsf = [&](const void* src, size_t n, uint4* dst) {
+        return cuda_status(launch_weight_sf(static_cast<const float*>(src), n, dst, status, s));
+      };
+      if (st == MOE_OK) st = wsf(wts->w13_s, E * n13, wsf13);
+      if (st == MOE_OK) st = wsf(wts->w2_s, E * n2, wsf2);
+      if (st == MOE_OK && S > 0) st = wsf(wts->ws13_s, S * n13, wsf13 + E * n13);
+      if (st == MOE_OK && S > 0) st = wsf(wts->ws2_s, S * n2, wsf2 + E * n2);
+    }
     if (st != MOE_OK) return st;
     x_router = at<void>(ws, L.x_bf16);
   }
@@ -624,11 +671,20 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if ((st = mark(4)) != MOE_OK) return st;
   void* y_rows = at<void>(ws, L.y_rows);
   if (fp8) {
-    const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
-    const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
-    st = run_ffn_fp8(c, L, ws, x_perm, x_perm_sf, R, w13_b, w2_b, wsf13, wsf2, E, x_b, x_sf, T, ws13_b,
-                     ws2_b, wsf13 + E * n13, wsf2 + E * n2, S, L.rows_all, y_rows, chunk_rows, s,
-                     ev ? ev + 5 : nullptr);
+    Fp8Seg s0{x_perm, x_perm_sf, R, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E};
+    Fp8Seg s1{x_b, x_sf, T, ws13_b, ws2_b, nullptr, nullptr, nullptr, nullptr, S};
+    if (w4) {
+      s0.wsc13 = static_cast<const uint8_t*>(wts->w13_s);
+      s0.wsc2 = static_cast<const uint8_t*>(wts->w2_s);
+      s1.wsc13 = static_cast<const uint8_t*>(wts->ws13_s);
+      s1.wsc2 = static_cast<const uint8_t*>(wts->ws2_s);
+    } else {
+      s0.wsf13 = wsf13;
+      s0.wsf2 = wsf2;
+      s1.wsf13 = wsf13 + E * n13;
+      s1.wsf2 = wsf2 + E * n2;
+    }
+    st = run_ffn_fp8(c, L, ws, s0, s1, L.rows_all, y_rows, chunk_rows, s, ev ? ev + 5 : nullptr);
   } else {
     st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows,
                  chunk_rows, s, ev ? ev + 5 : nullptr);

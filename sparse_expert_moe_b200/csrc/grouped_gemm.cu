@@ -75,6 +75,8 @@ struct DevParams {
   int* status;
   // FP8 block scaling
   const uint4* wsf[2];        // [groups][row blocks][k blocks] UE8M0 x16 per 128x128 weight block
+  const uint8_t* wsc[2];      // FP4 weights: E8M0 code per row per 32 K-elements [rows][K / 32]
+  int wsc_ld;                 // K / 32
   int wsf_rb_per_group;       // 128-row blocks of the weight matrix per group
   const uint32_t* tsf[2];     // [k blocks][rows] UE8M0 x4 per (128-element block, token row)
   int tsf_ld[2];
@@ -91,8 +93,13 @@ struct DevParams {
 // the single-block FFN2 used when d_model is not a multiple of 256.
 template <int MODE, int NTW = kChunkRows>
 struct Cfg {
-  static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8;
-  static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8;   // gate + up accumulators
+  // FP4 weights (MXFP4: E2M1, one E8M0 scale per 32 K-elements) with e4m3 tokens: the FP8
+  // kernel with the weight operand unpacked by TMA into the e4m3 layout
+  static constexpr bool kW4 = MODE == kFFN1F4 || MODE == kFFN2F4;
+  static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8 || kW4;
+  static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8 || MODE == kFFN1F4;  // gate + up
+  static constexpr bool kSecond = MODE == kFFN2 || MODE == kFFN2M256 || MODE == kFFN2M512 ||
+                                  MODE == kFFN2F8 || MODE == kFFN2F4;   // reads h (output rows)
   // FFN2: 128-row weight blocks (= 128 output columns each) per tile
   static constexpr int kOutBlocks = MODE == kFFN2M512 ? 4 : (MODE == kFFN2M256 ? 2 : 1);
   static_assert(NTW == kChunkRows || MODE != kRouter, "router tiles are 128 tokens wide");
@@ -364,9 +371,10 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
         const int a_row = c.group * p.w_rows_per_group + mb * kBM * C::kOutBlocks;
         const int n_pad = (c.nrows + 15) & ~15;
         // the second GEMM reads the h rows the first one wrote (output numbering)
-        const int tok_row = (MODE == kFFN2 || MODE == kFFN2M256 || MODE == kFFN2M512 || MODE == kFFN2F8)
-                                ? c.o_row : c.b_row;
-        const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;   // TMA bytes per stage
+        const int tok_row = C::kSecond ? c.o_row : c.b_row;
+        // TMA bytes per stage: a packed FP4 weight box lands unpacked (16 KB of shared memory)
+        // but completes its packed size in bytes (8 KB) on the barrier
+        const uint32_t bytes = C::kATiles * (C::kW4 ? kABytes / 2 : kABytes) + n_pad * kRowBytes;
         const uint32_t stage_bytes = C::kFP8 ? C::kStageBytes : bytes;     // ring bytes per stage
         const CUtensorMap* wm = &p.wmap[c.seg];
         for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
@@ -409,6 +417,8 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
         if (c.nrows <= 0) continue;
         const int n_pad = (c.nrows + 15) & ~15;
         const uint32_t idesc = C::kFP8 ? idesc_e4m3_bs(kBM, n_pad) : idesc_bf16_f32(kBM, n_pad);
+        // FP4 weights: MMA kk of a stage applies byte kk of each weight row's scale word
+        const uint32_t idesc_w4 = idesc_mx_bs(kFmtE2M1, kFmtE4M3, kBM, n_pad, 0, 0);
         const uint32_t acc = it % C::kAccBufs;
         const uint32_t acc_phase = (it / C::kAccBufs) & 1;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
@@ -440,9 +450,10 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
               const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
-              umma_e4m3_bs(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, sfa, sfb, accum);
+              const uint32_t id = C::kW4 ? (idesc_w4 | (static_cast<uint32_t>(kk) << 29)) : idesc;
+              umma_e4m3_bs(d0, umma_desc_sw128(st + kk * 32), bdesc, id, sfa, sfb, accum);
               if (C::kGLU)
-                umma_e4m3_bs(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, idesc, sfa + 4, sfb,
+                umma_e4m3_bs(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, id, sfa + 4, sfb,
                              accum);
             }
           } else {
@@ -486,7 +497,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + acc * C::kAccCols;
       const int m = mb * kBM + m_local;       // output column
-      if (MODE == kFFN1F8) {
+      if (C::kGLU && C::kFP8) {
         // SwiGLU, then requantise h to e4m3 with one power-of-two scale per token per 128
         // h columns (this tile's columns).  Pass 1: per token, the maximum |h| of each
         // warp's 32 columns (redux.sync) into shared memory; one exchange between the
@@ -532,7 +543,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
         }
         rbuf ^= 1u;
       }
-      for (int n0 = 0; n0 < c.nrows && MODE != kFFN1F8; n0 += 16) {
+      for (int n0 = 0; n0 < c.nrows && !(C::kGLU && C::kFP8); n0 += 16) {
         if (MODE == kFFN1) {
           float g[16], u[16];
           tmem_ld16x2(tb + n0, tb + C::kNT + n0, g, u);
@@ -561,7 +572,7 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
             store_block_16x32(yrow + (j + 1) * kBM, p.ld_out, c.nrows - n0, yv,
                               reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
           }
-        } else if (MODE == kFFN2 || MODE == kFFN2F8) {
+        } else if (MODE == kFFN2 || MODE == kFFN2F8 || MODE == kFFN2F4) {
           float v[16];
           tmem_ld16(tb + n0, v);
           __nv_bfloat16 yv[16];
@@ -588,10 +599,12 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
     }
   } else if (C::kFP8) {
     // ------------------------------------------------------------ scale-factor warp (FP8)
-    // Per stage: the 512-byte scale atoms of the weight tile(s) (one UE8M0 value for the
-    // whole 128x128 block, replicated) and of the token rows (row n's 4 bytes at
-    // (n % 32) * 16 + (n / 32) * 4), copied with cp.async; each lane's completion
-    // arrives on the stage's full barrier.
+    // Per stage: the 512-byte scale atoms of the weight tile(s) and of the token rows (row
+    // n's 4 bytes at (n % 32) * 16 + (n / 32) * 4), copied with cp.async; each lane's
+    // completion arrives on the stage's full barrier.  e4m3 weights: one UE8M0 value for
+    // the whole 128x128 block, replicated.  FP4 weights: row r's 4 bytes are its E8M0
+    // scales of the stage's four 32-element K runs, read straight from the caller's
+    // [rows][K / 32] codes.
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     const int up_rb = p.up_offset / kBM;
@@ -601,8 +614,9 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
       if (c.nrows <= 0) continue;
       const int mb = tc.mb;
       const int n_pad = (c.nrows + 15) & ~15;
-      const int tok_row = MODE == kFFN2F8 ? c.o_row : c.b_row;
-      const uint4* wsf = p.wsf[c.seg] + static_cast<size_t>(c.group) * p.wsf_rb_per_group * p.k_blocks;
+      const int tok_row = C::kSecond ? c.o_row : c.b_row;
+      const uint4* wsf = C::kW4 ? nullptr
+                                : p.wsf[c.seg] + static_cast<size_t>(c.group) * p.wsf_rb_per_group * p.k_blocks;
       const uint32_t* tsf = p.tsf[c.seg];
       const int tld = p.tsf_ld[c.seg], trows = p.tsf_rows[c.seg];
       for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
@@ -612,9 +626,22 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           break;
         }
         uint8_t* sf = tiles + stage * C::kStageBytes + C::kATiles * kABytes + C::kBBytes;
-        cp_async_16(sf + lane * 16, wsf + static_cast<size_t>(mb) * p.k_blocks + kb);
-        if (C::kGLU)
-          cp_async_16(sf + kSFAtomBytes + lane * 16, wsf + static_cast<size_t>(up_rb + mb) * p.k_blocks + kb);
+        if (C::kW4) {
+          const uint8_t* wsc = p.wsc[c.seg] +
+              (static_cast<size_t>(c.group) * p.w_rows_per_group + mb * kBM) * p.wsc_ld + kb * 4;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            cp_async_4(sf + lane * 16 + j * 4, wsc + static_cast<size_t>(j * 32 + lane) * p.wsc_ld);
+            if (C::kGLU)
+              cp_async_4(sf + kSFAtomBytes + lane * 16 + j * 4,
+                         wsc + static_cast<size_t>(p.up_offset + j * 32 + lane) * p.wsc_ld);
+          }
+        } else {
+          cp_async_16(sf + lane * 16, wsf + static_cast<size_t>(mb) * p.k_blocks + kb);
+          if (C::kGLU)
+            cp_async_16(sf + kSFAtomBytes + lane * 16,
+                        wsf + static_cast<size_t>(up_rb + mb) * p.k_blocks + kb);
+        }
         uint8_t* sfb = sf + C::kATiles * kSFAtomBytes;
 #pragma unroll
         for (int j = 0; j < 4 * C::kSFBAtoms; ++j) {
@@ -792,11 +819,13 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   p.status = g.status;
   for (int i = 0; i < 2; ++i) {
     p.wsf[i] = g.wsf[i];
+    p.wsc[i] = g.wsc[i];
     p.tsf[i] = g.tsf[i];
     p.tsf_ld[i] = g.tsf_ld[i];
     p.tsf_rows[i] = g.tsf_rows[i];
   }
   p.wsf_rb_per_group = g.wsf_rb_per_group;
+  p.wsc_ld = g.wsc_ld;
   p.out_sf = g.out_sf;
   p.ld_out_sf = g.ld_out_sf;
   cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, NTW>,
@@ -826,10 +855,22 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
     case kFFN2:   // d_model not a multiple of 256: one 128-row weight block per tile
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2, kChunkRowsNarrow>(g, s);
       return launch_mode<kFFN2, kChunkRowsWide>(g, s);
-    case kFFN1F8: return launch_mode<kFFN1F8, kChunkRows>(g, s);
+    // FP8 / FP4-weight tiles: 32 tokens (decode-sized batches), else 112 (kChunkRows maps to
+    // kChunkRowsFP8); the second GEMM takes 224-token tiles once chunks are 224 rows
+    case kFFN1F8:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1F8, kChunkRowsNarrow>(g, s);
+      return launch_mode<kFFN1F8, kChunkRows>(g, s);
     case kFFN2F8:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2F8, kChunkRowsNarrow>(g, s);
       if (g.tile_tokens == 2 * kChunkRowsFP8) return launch_mode<kFFN2F8, 2 * kChunkRowsFP8>(g, s);
       return launch_mode<kFFN2F8, kChunkRows>(g, s);
+    case kFFN1F4:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1F4, kChunkRowsNarrow>(g, s);
+      return launch_mode<kFFN1F4, kChunkRows>(g, s);
+    case kFFN2F4:
+      if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2F4, kChunkRowsNarrow>(g, s);
+      if (g.tile_tokens == 2 * kChunkRowsFP8) return launch_mode<kFFN2F4, 2 * kChunkRowsFP8>(g, s);
+      return launch_mode<kFFN2F4, kChunkRows>(g, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -79,9 +79,10 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
                         int32_t* grp_cp, int32_t* n_grp, int* status, cudaStream_t s);
 
 // kFFN2M256 / kFFN2M512: FFN2 (bf16) with 256 / 512 weight rows per tile, as two / four
-// 128-row blocks (M512: decode-sized token tiles only).
+// 128-row blocks (M512: decode-sized token tiles only).  kFFN1F4 / kFFN2F4: the FP8 GEMMs
+// with FP4 (MXFP4) weights.
 enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5,
-                kFFN2M512 = 6 };
+                kFFN2M512 = 6, kFFN1F4 = 7, kFFN2F4 = 8 };
 
 struct GemmLaunch {
   int mode;
@@ -112,6 +113,9 @@ struct GemmLaunch {
   // the scales of its requantised output to out_sf ([I / 128][ld_out_sf]).
   const uint4* wsf[2];
   int wsf_rb_per_group;
+  // FP4 modes: E8M0 weight scale codes per segment, [rows][K / 32] (wsc_ld = K / 32)
+  const uint8_t* wsc[2];
+  int wsc_ld;
   const uint32_t* tsf[2];
   int tsf_ld[2];
   int tsf_rows[2];
@@ -127,6 +131,12 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 // Same for 1-byte (e4m3) elements, box {128 columns, box_rows rows}.
 bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                   uint32_t box_rows);
+// Packed FP4 (two E2M1 codes per byte, `cols` elements per row), box {128 elements,
+// box_rows rows}, loaded into shared memory unpacked to one 16-byte slot per 16 elements
+// (8 data bytes, 8 bytes of gap): the e4m3 tile layout the block-scaled MMA reads FP4
+// operands from.  Needs a 32-byte aligned base and cols a multiple of 128.
+bool make_tmap_fp4(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows);
 
 // FP8 preparation kernels.
 // x e4m3 [T, d] + x_scale fp32 [T, d/128] -> x_bf16 [T, d] (exact) and x_sf [d/128][T]

@@ -254,11 +254,23 @@ __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t 
                : "memory");
 }
 
-// Instruction descriptor of kind::mxf8f6f4 with block scaling: e4m3 A and B
-// (format 0), both K-major, UE8M0 scale factors (bit 23), shape M x N, scale
-// factor ids 0.
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: A and B element formats
+// (bits 7-9 / 10-12: 0 = E4M3, 5 = E2M1), both K-major, UE8M0 scale factors (bit 23),
+// shape M x N.  Each MMA covers 32 K-elements and applies one scale per row of A and of B;
+// a_sf (bits 29-30) / b_sf (bits 4-5) select which byte of the row's 32-bit scale word in
+// TMEM that is.
+__host__ __device__ constexpr uint32_t idesc_mx_bs(int a_fmt, int b_fmt, int M, int N, int a_sf,
+                                                   int b_sf) {
+  return (static_cast<uint32_t>(b_sf) << 4) | (static_cast<uint32_t>(a_fmt) << 7) |
+         (static_cast<uint32_t>(b_fmt) << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(a_sf) << 29);
+}
+constexpr int kFmtE4M3 = 0;
+constexpr int kFmtE2M1 = 5;
+
+// e4m3 A and B, scale byte 0 (the FP8 path's scales are replicated across the word).
 __host__ __device__ constexpr uint32_t idesc_e4m3_bs(int M, int N) {
-  return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
+  return idesc_mx_bs(kFmtE4M3, kFmtE4M3, M, N, 0, 0);
 }
 
 // D[tmem] (+)= (A * sfa) x (B * sfb)^T over K = 32 e4m3 elements, one scale per

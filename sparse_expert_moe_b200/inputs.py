@@ -21,10 +21,15 @@ More, Smaller Experts" -- 384 experts, top-8 plus one shared expert):
 
   tiny            T=64   d=128  E=8   k=2 I=256  S=0 softmax       fp32
   r1_decode       T=128  d=7168 E=256 k=8 I=2048 S=1 sigmoid+bias  bf16
+  r1_decode_uniform  r1_decode's activations with no selection bias: uniform routing,
+                  about 252 of the 256 experts touched per batch
   r1_prefill      T=8192 d=7168 E=256 k=8 I=2048 S=1 sigmoid+bias  bf16, Zipf(1.1) loads
   kimi            T=4096 d=7168 E=384 k=8 I=2048 S=1 sigmoid+bias  bf16
   r1_prefill_fp8  r1_prefill with e4m3 activations (1x128 scales) and e4m3
                   weights (128x128 scales), bf16 output
+  r1_decode_fp8   r1_decode with e4m3 activations and e4m3 weights
+  r1_decode_fp4   r1_decode with e4m3 activations and MXFP4 weights (E2M1 codes, one E8M0
+                  scale per 32 elements along K)
 """
 from __future__ import annotations
 
@@ -74,10 +79,16 @@ SPECS = {
                  family="tiny", x_stream=1, margin=1e-2),
     "r1_decode": Spec("r1_decode", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "bf16", "bf16",
                       "bf16", family="r1", x_stream=2, bias_range=0.1),
+    "r1_decode_uniform": Spec("r1_decode_uniform", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias",
+                              "bf16", "bf16", "bf16", family="r1", x_stream=2),
     "r1_prefill": Spec("r1_prefill", 8192, 7168, 256, 8, 2048, 1, "sigmoid_bias", "bf16", "bf16",
                        "bf16", family="r1", x_stream=3, loads="zipf"),
     "kimi": Spec("kimi", 4096, 7168, 384, 8, 2048, 1, "sigmoid_bias", "bf16", "bf16", "bf16",
                  family="kimi", x_stream=4),
+    "r1_decode_fp8": Spec("r1_decode_fp8", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
+                          "e4m3", "bf16", family="r1", x_stream=2, bias_range=0.1),
+    "r1_decode_fp4": Spec("r1_decode_fp4", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
+                          "e2m1", "bf16", family="r1", x_stream=2, bias_range=0.1),
     "r1_prefill_fp8": Spec("r1_prefill_fp8", 8192, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
                            "e4m3", "bf16", family="r1", x_stream=3, loads="zipf"),
 }
@@ -126,6 +137,29 @@ def to_e4m3_blocks(a: np.ndarray, br: int, bc: int):
     return q, torch.from_numpy(s)
 
 
+E2M1_MAX = 6.0
+
+
+def to_mxfp4(a: np.ndarray, block: int = 32):
+    """fp32 draw [R, C] -> MXFP4: (packed E2M1 codes as uint8 [R, C/2], the even element in
+    the low nibble; E8M0 scale codes as uint8 [R, C/block]).
+
+    Each 1 x block run along C shares the smallest power-of-two scale s with amax / s <= 6
+    (E2M1's largest magnitude; 1.0 for an all-zero block); the elements a / s are rounded
+    to the nearest E2M1 value, ties to even (ml_dtypes' float4_e2m1fn conversion)."""
+    import ml_dtypes
+    R, C = a.shape
+    amax = np.abs(a).reshape(R, C // block, block).max(axis=2)
+    v = np.asarray(amax, np.float64) / E2M1_MAX
+    m, e = np.frexp(v)
+    e = np.where(m == 0.5, e - 1, e)                    # exact powers of two
+    e = np.where(v > 0, e, 0)
+    q = (np.asarray(a, np.float32) / np.repeat(np.ldexp(1.0, e), block, axis=1).astype(np.float32))
+    codes = q.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return torch.from_numpy(packed), torch.from_numpy((e + 127).astype(np.uint8))
+
+
 # ---------------------------------------------------------------------------
 # draws
 # ---------------------------------------------------------------------------
@@ -161,6 +195,8 @@ def _encode_weight(spec: Spec, w32: np.ndarray):
         return to_bf16(w32), None
     if spec.weight == "e4m3":
         return to_e4m3_blocks(w32, 128, 128)
+    if spec.weight == "e2m1":
+        return to_mxfp4(w32)
     raise ValueError(spec.weight)
 
 
@@ -246,12 +282,19 @@ class Workload:
 
 def _stack_experts(spec, seed, n, shared, threads):
     I, d = spec.d_ff, spec.d_model
-    wdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[spec.weight]
-    w13 = torch.empty((n, 2 * I, d), dtype=wdt)
-    w2 = torch.empty((n, d, I), dtype=wdt)
-    scaled = spec.weight == "e4m3"
-    s13 = torch.empty((n, 2 * I // 128, d // 128), dtype=torch.float32) if scaled else None
-    s2 = torch.empty((n, d // 128, I // 128), dtype=torch.float32) if scaled else None
+    if spec.weight == "e2m1":          # packed codes [rows, K/2] + E8M0 codes [rows, K/32]
+        w13 = torch.empty((n, 2 * I, d // 2), dtype=torch.uint8)
+        w2 = torch.empty((n, d, I // 2), dtype=torch.uint8)
+        s13 = torch.empty((n, 2 * I, d // 32), dtype=torch.uint8)
+        s2 = torch.empty((n, d, I // 32), dtype=torch.uint8)
+        scaled = True
+    else:
+        wdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[spec.weight]
+        w13 = torch.empty((n, 2 * I, d), dtype=wdt)
+        w2 = torch.empty((n, d, I), dtype=wdt)
+        scaled = spec.weight == "e4m3"
+        s13 = torch.empty((n, 2 * I // 128, d // 128), dtype=torch.float32) if scaled else None
+        s2 = torch.empty((n, d // 128, I // 128), dtype=torch.float32) if scaled else None
 
     def one(e):
         q13, a13, q2, a2 = draw_expert(spec, seed, e, shared)

@@ -66,10 +66,74 @@ def margin_workload(spec, seed=0, threads=None):
     return inputs.make_workload(spec, seed, redraw=sorted(attempts.items()), threads=threads)
 
 
+_E4M3_TABLE = None
+
+
+def dequant_fast(codes, scales, br, bc):
+    """oracle.dequantize_blocks by table lookup: the oracle's decoding of all 256 e4m3 codes,
+    indexed by the codes, times each block's scale (broadcast, no repeated scale array).
+    Equal to oracle.dequantize_blocks bit for bit (tests/test_oracle_pins.py checks it);
+    used where whole expert weight sets are decoded, to keep the oracle runs short."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        _E4M3_TABLE = oracle.decode_e4m3(np.arange(256, dtype=np.uint8))
+    c = np.asarray(codes, np.uint8)
+    R, C = c.shape
+    v = _E4M3_TABLE[c].reshape(R // br, br, C // bc, bc)
+    v *= np.asarray(scales, np.float64)[:, None, :, None]
+    return v.reshape(R, C)
+
+
+_FP4_TABLE = None
+
+
+def dequant_mxfp4_fast(packed, scale_codes):
+    """oracle.dequantize_mxfp4 by table lookup: the oracle's decoding of both nibbles of
+    all 256 bytes, indexed by the packed bytes, times each 32-element run's decoded E8M0
+    scale (broadcast).  Equal to the oracle bit for bit (tests/test_oracle_pins.py)."""
+    global _FP4_TABLE
+    if _FP4_TABLE is None:
+        _FP4_TABLE = oracle.decode_e2m1(oracle.unpack_fp4(np.arange(256, dtype=np.uint8)[:, None]))
+    p = np.asarray(packed, np.uint8)
+    R, half = p.shape
+    v = _FP4_TABLE[p].reshape(R, 2 * half // 32, 32)
+    v *= oracle.decode_e8m0(scale_codes)[:, :, None]
+    return v.reshape(R, 2 * half)
+
+
 def _w_values(w, s, shape_blocks):
     if s is None:
         return w.double().numpy()
-    return oracle.dequantize_blocks(w.view(torch.uint8).numpy(), s.numpy(), 128, 128)
+    if s.dtype == torch.uint8:          # MXFP4: packed E2M1 + E8M0 codes
+        return dequant_mxfp4_fast(w.numpy(), s.numpy())
+    return dequant_fast(w.view(torch.uint8).numpy(), s.numpy(), 128, 128)
+
+
+def oracle_routing(wl):
+    """The oracle's router, top-k and permutation over every token of workload wl."""
+    spec = wl.spec
+    logits = oracle.router_logits(act_values(wl), wl.wr.double().numpy())
+    bias = None if wl.sel_bias is None else wl.sel_bias.double().numpy()
+    idx, gates = oracle.route(logits, spec.score, spec.top_k, bias)
+    offsets, perm_token, inv_perm = oracle.permute(idx, spec.E)
+    return dict(idx=idx, gates=gates, offsets=offsets, perm_token=perm_token, inv_perm=inv_perm)
+
+
+def tile_edge_tokens(routing, T, n_shared, unit):
+    """Tokens holding the first and the last row of every `unit`-row piece of every routed
+    group (the GEMM tiles' token ranges: every group's first and last chunk among them),
+    and of the shared experts' T rows."""
+    off, pt = routing["offsets"], routing["perm_token"]
+    rows = []
+    for e in range(len(off) - 1):
+        lo, hi = int(off[e]), int(off[e + 1])
+        for s in range(lo, hi, unit):
+            rows += [s, min(s + unit, hi) - 1]
+    toks = set(pt[np.asarray(rows, np.int64)].tolist()) if rows else set()
+    if n_shared:
+        for s in range(0, T, unit):
+            toks.update((s, min(s + unit, T) - 1))
+    return np.array(sorted(toks), np.int64)
 
 
 def oracle_layer(wl, rows=None, return_routing=False):

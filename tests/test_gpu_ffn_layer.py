@@ -9,7 +9,7 @@ import torch
 import oracle
 from sparse_expert_moe_b200 import inputs, moe
 
-from helpers import margin_workload, max_rel_err, oracle_layer
+from helpers import margin_workload, max_rel_err, oracle_layer, oracle_routing, tile_edge_tokens
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -55,6 +55,45 @@ def test_grouped_ffn_vs_oracle(sizes, d, I):
     got = y.float().cpu().numpy()
     assert np.isfinite(got).all()
     assert max_rel_err(got, ref) < TOL_BF16
+
+
+def row_rel_err(y, ref):
+    """Per row: ||y_r - ref_r||_inf / ||ref_r||_inf."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return np.abs(y - ref).max(axis=1) / np.maximum(np.abs(ref).max(axis=1), 1e-30)
+
+
+@pytest.mark.slow
+def test_grouped_ffn_r1_shape_every_row():
+    """The DeepSeek-R1 expert shape (d = 7168, I = 2048: 112 K blocks in the first GEMM, 32 in
+    the second) on groups that take every path of the tile scheduler: a Zipf-head group of
+    7300 rows (29 chunks of 256 rows, a ragged last chunk whose second half holds 4 rows),
+    one of 257 rows (a full chunk and a 1-row chunk), one of 1 row and an empty one.  Every
+    output row is compared with the oracle."""
+    sizes, d, I = [7300, 257, 1, 0], 7168, 2048
+    rng = np.random.default_rng(71)
+    G, n_rows = len(sizes), sum(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    a = _bf16(rng.standard_normal((n_rows, d), dtype=np.float32))
+    w13 = _bf16(rng.standard_normal((G, 2 * I, d), dtype=np.float32) * np.float32(0.02))
+    w2 = _bf16(rng.standard_normal((G, d, I), dtype=np.float32) * np.float32(0.02))
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0)
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows, a.to(DEV), None,
+                        w13.to(DEV), None, w2.to(DEV), None, y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    for g in range(G):
+        lo, hi = offsets[g], offsets[g + 1]
+        if hi == lo:
+            continue
+        ref = oracle.swiglu_expert(a[lo:hi].double().numpy(), w13[g].double().numpy(),
+                                   w2[g].double().numpy())
+        assert max_rel_err(got[lo:hi], ref) < TOL_BF16, g
+        assert row_rel_err(got[lo:hi], ref).max() < TOL_BF16, g
 
 
 def test_grouped_ffn_all_groups_empty():
@@ -139,7 +178,13 @@ def _run_layer(wl, T=None):
 
 
 def _check_layer(wl, rows=None):
+    """The layer against the oracle: routing of every token bit-exact (indices) and within
+    1e-5 (gates); outputs of every token, or of the sampled `rows`, within the bar."""
     layer, y, idx, gw = _run_layer(wl)
+    if rows is not None:
+        full = oracle_routing(wl)
+        assert np.array_equal(idx, full["idx"])
+        np.testing.assert_allclose(gw, full["gates"], rtol=1e-5, atol=1e-6)
     ref, r = oracle_layer(wl, rows=rows, return_routing=True)
     if rows is not None:
         y, idx, gw = y[rows], idx[rows], gw[rows]
@@ -197,18 +242,23 @@ def _full_workload(name):
 
 
 @pytest.mark.slow
-def test_layer_r1_decode_full():
-    """The DeepSeek-R1-shaped decode layer, every token checked."""
-    wl = _full_workload("r1_decode")
+@pytest.mark.parametrize("name", ["r1_decode", "r1_decode_uniform"])
+def test_layer_r1_decode_full(name):
+    """The DeepSeek-R1-shaped decode layer, every token checked: with the stated selection
+    bias (143 experts touched) and uniformly routed (252 experts touched)."""
+    wl = _full_workload(name)
     _check_layer(wl)
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["r1_prefill", "kimi"])
 def test_layer_full_size_sampled(name):
-    """Full-size prefill-shaped layers in the launch configuration the bench times; the
-    oracle evaluates a sample of tokens one by one (the layer is per-token)."""
+    """Full-size prefill-shaped layers in the launch configuration the bench times.  The
+    routing of every token is compared; the oracle evaluates the outputs of the tokens that
+    hold the first and the last row of every 128-row token tile of every expert group
+    (every group's first and last chunk among them) -- the layer is per-token, so these
+    are exact comparisons of those tokens."""
     wl = _full_workload(name)
-    rng = np.random.default_rng(0)
-    rows = np.sort(rng.choice(wl.spec.T, 12, replace=False))
+    rows = tile_edge_tokens(oracle_routing(wl), wl.spec.T, wl.spec.n_shared, 128)
+    assert rows.size >= 256
     _check_layer(wl, rows=rows)

@@ -8,7 +8,8 @@ import torch
 import oracle
 from sparse_expert_moe_b200 import inputs, moe
 
-from helpers import margin_workload, max_rel_err, oracle_layer
+from helpers import (dequant_fast, dequant_mxfp4_fast, margin_workload, max_rel_err, oracle_layer,
+                     oracle_routing, tile_edge_tokens)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -58,6 +59,90 @@ def test_grouped_ffn_fp8_vs_oracle(sizes, d, I):
     assert max_rel_err(got, ref) < TOL_FP8
 
 
+@pytest.mark.slow
+def test_grouped_ffn_fp8_r1_shape_every_row():
+    """FP8 at the DeepSeek-R1 expert shape (d = 7168, I = 2048: 56 K blocks of 128 in the
+    first GEMM, 16 in the second): a 7300-row group (33 chunks of 224 rows; the first GEMM
+    takes them as 112-row halves, the last chunk's second half holding 20 rows), one of 257
+    rows (224 + 33), one of 1 row and an empty one.  Every output row is compared with the
+    oracle on the decoded inputs."""
+    sizes, d, I = [7300, 257, 1, 0], 7168, 2048
+    rng = np.random.default_rng(72)
+    G, n_rows = len(sizes), sum(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    a, a_s = _e4m3(rng.standard_normal((n_rows, d), dtype=np.float32), 1, 128)
+    w13 = [_e4m3(rng.standard_normal((2 * I, d), dtype=np.float32) * np.float32(0.02), 128, 128)
+           for _ in range(G)]
+    w2 = [_e4m3(rng.standard_normal((d, I), dtype=np.float32) * np.float32(0.02), 128, 128)
+          for _ in range(G)]
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0, act="e4m3", weight="e4m3")
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows,
+                        a.view(torch.uint8).to(DEV), a_s.to(DEV),
+                        torch.stack([q for q, _ in w13]).to(DEV), torch.stack([s for _, s in w13]).to(DEV),
+                        torch.stack([q for q, _ in w2]).to(DEV), torch.stack([s for _, s in w2]).to(DEV),
+                        y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    av = dequant_fast(a.view(torch.uint8).numpy(), a_s.numpy(), 1, 128)
+    for g in range(G):
+        lo, hi = offsets[g], offsets[g + 1]
+        if hi == lo:
+            continue
+        ref = oracle.swiglu_expert(av[lo:hi], dequant_fast(w13[g][0].view(torch.uint8).numpy(),
+                                                           w13[g][1].numpy(), 128, 128),
+                                   dequant_fast(w2[g][0].view(torch.uint8).numpy(),
+                                                w2[g][1].numpy(), 128, 128))
+        assert max_rel_err(got[lo:hi], ref) < TOL_FP8, g
+        # per row: h is requantised to e4m3 (3 mantissa bits), so single rows scatter more
+        # than the whole output; twice the bar still exposes a wrong tile or chunk
+        row = np.abs(got[lo:hi] - ref).max(axis=1) / np.abs(ref).max(axis=1)
+        assert row.max() < 2 * TOL_FP8, g
+
+
+def _mxfp4(rows, cols, rng, std=0.05):
+    """MXFP4 weights whose 32-element runs differ in magnitude by up to 2^6, so that every
+    run needs its own E8M0 scale (a scale applied to the wrong run shows in the output)."""
+    w = rng.standard_normal((rows, cols)) * std * np.exp2(rng.integers(-3, 4, (rows, cols // 32))).repeat(32, 1)
+    return inputs.to_mxfp4(w.astype(np.float32))
+
+
+@pytest.mark.parametrize("sizes,d,I", [
+    ([5, 0, 1, 130, 16, 17, 0, 112], 256, 256),     # 112 / 224-row tiles, ragged, empty
+    ([300], 128, 384),
+    ([1, 2, 3], 512, 128),                           # decode-sized: 32-token tiles
+    ([3, 0, 17, 32, 33], 1024, 256),
+])
+def test_grouped_ffn_fp4_weights_vs_oracle(sizes, d, I):
+    """FP4 (MXFP4) expert weights with e4m3 token rows; h requantised to e4m3."""
+    rng = np.random.default_rng(sum(sizes) + d + 1)
+    G, n_rows = len(sizes), sum(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    a, a_s = _e4m3(rng.standard_normal((n_rows, d)) * np.exp2(rng.integers(-3, 3, (n_rows, 1))), 1, 128)
+    w13 = [_mxfp4(2 * I, d, rng) for _ in range(G)]
+    w2 = [_mxfp4(d, I, rng) for _ in range(G)]
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0, act="e4m3", weight="e2m1")
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows, a.view(torch.uint8).to(DEV),
+                        a_s.to(DEV), torch.stack([q for q, _ in w13]).to(DEV),
+                        torch.stack([s for _, s in w13]).to(DEV), torch.stack([q for q, _ in w2]).to(DEV),
+                        torch.stack([s for _, s in w2]).to(DEV), y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    av = _dq(a, a_s, 1, 128)
+    ref = np.zeros((n_rows, d))
+    for g in range(G):
+        lo, hi = offsets[g], offsets[g + 1]
+        if hi > lo:
+            ref[lo:hi] = oracle.swiglu_expert(av[lo:hi], oracle.dequantize_mxfp4(*[t.numpy() for t in w13[g]]),
+                                              oracle.dequantize_mxfp4(*[t.numpy() for t in w2[g]]))
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert max_rel_err(got, ref) < TOL_FP8
+
+
 def test_permute_fp8_rows_and_scales():
     T, E, k, d = 300, 32, 4, 256
     rng = np.random.default_rng(9)
@@ -82,7 +167,7 @@ def test_permute_fp8_rows_and_scales():
     assert torch.equal(x_perm_s.cpu(), xs[tp])
 
 
-def _check_fp8_layer(wl, rows=None):
+def _check_fp8_layer(wl, rows=None, routing=None):
     layer = moe.DeviceLayer.from_workload(wl, DEV)
     idx = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.int32, device=DEV)
     gw = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.float32, device=DEV)
@@ -90,6 +175,10 @@ def _check_fp8_layer(wl, rows=None):
     torch.cuda.synchronize()
     assert moe.moe_read_device_status(layer.ws) == 0
     got, idx, gw = y.float().cpu().numpy(), idx.cpu().numpy(), gw.cpu().numpy()
+    del layer
+    if routing is not None:
+        assert np.array_equal(idx, routing["idx"])
+        np.testing.assert_allclose(gw, routing["gates"], rtol=1e-5, atol=1e-6)
     ref, r = oracle_layer(wl, rows=rows, return_routing=True)
     if rows is not None:
         got, idx, gw = got[rows], idx[rows], gw[rows]
@@ -101,9 +190,19 @@ def _check_fp8_layer(wl, rows=None):
 
 @pytest.mark.parametrize("T,d,E,k,I,S", [(70, 256, 16, 4, 256, 1), (300, 384, 8, 2, 128, 2),
                                          (1, 128, 4, 1, 128, 1)])
-def test_layer_fp8_custom(T, d, E, k, I, S):
-    spec = inputs.custom_spec(T, d, E, k, I, S, act="e4m3", weight="e4m3")
+@pytest.mark.parametrize("weight", ["e4m3", "e2m1"])
+def test_layer_fp8_custom(T, d, E, k, I, S, weight):
+    spec = inputs.custom_spec(T, d, E, k, I, S, act="e4m3", weight=weight)
     _check_fp8_layer(margin_workload(spec, seed=T + 1))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["r1_decode_fp8", "r1_decode_fp4"])
+def test_layer_r1_decode_low_precision_full(name):
+    """The DeepSeek-R1 decode layer with e4m3 activations and e4m3 or MXFP4 weights, every
+    token checked."""
+    wl = inputs.load_workload(name)
+    _check_fp8_layer(wl, routing=oracle_routing(wl))
 
 
 @pytest.mark.parametrize("which,value", [("w13_s", 0.75), ("w2_s", 0.0), ("ws2_s", -0.5),
@@ -138,6 +237,10 @@ def test_layer_fp8_scale_outside_ue8m0_sets_device_status(which, value):
 
 @pytest.mark.slow
 def test_layer_fp8_full_size_sampled():
+    """The full-size FP8 prefill layer: routing of every token; outputs of the tokens holding
+    the first and the last row of every 112-row token tile of every expert group."""
     wl = inputs.load_workload("r1_prefill_fp8")
-    rows = np.sort(np.random.default_rng(1).choice(wl.spec.T, 12, replace=False))
-    _check_fp8_layer(wl, rows=rows)
+    routing = oracle_routing(wl)
+    rows = tile_edge_tokens(routing, wl.spec.T, wl.spec.n_shared, 112)
+    assert rows.size >= 256
+    _check_fp8_layer(wl, rows=rows, routing=routing)

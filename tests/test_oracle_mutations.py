@@ -150,13 +150,27 @@ def _dequant_scales_transposed(q_codes, scales, block_rows, block_cols):
                                       block_rows, block_cols)
 
 
+def _e2m1_exponent_bias_0(codes):
+    return _REAL["decode_e2m1"](codes) * 2.0
+
+
+def _fp4_nibbles_swapped(packed):
+    out = _REAL["unpack_fp4"](packed)
+    return out.reshape(out.shape[:-1] + (-1, 2))[..., ::-1].reshape(out.shape)
+
+
+def _e8m0_bias_128(codes):
+    return _REAL["decode_e8m0"](codes) / 2.0
+
+
 def _router_logits_without_transpose(x, wr):
     x, wr = np.asarray(x, np.float64), np.asarray(wr, np.float64)
     return x @ wr.reshape(wr.shape[1], wr.shape[0])
 
 
 _REAL = {n: getattr(om, n) for n in ("gate_weights", "selection_keys", "combine", "decode_e4m3",
-                                      "dequantize_blocks")}
+                                      "dequantize_blocks", "decode_e2m1", "unpack_fp4",
+                                      "decode_e8m0")}
 
 MUTATIONS = [
     ("select_topk", _topk_ties_to_higher_index),
@@ -173,6 +187,9 @@ MUTATIONS = [
     ("decode_e4m3", _e4m3_exponent_bias_8),
     ("dequantize_blocks", _dequant_scales_transposed),
     ("router_logits", _router_logits_without_transpose),
+    ("decode_e2m1", _e2m1_exponent_bias_0),
+    ("unpack_fp4", _fp4_nibbles_swapped),
+    ("decode_e8m0", _e8m0_bias_128),
 ]
 
 

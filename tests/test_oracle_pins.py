@@ -113,6 +113,76 @@ def test_block_dequant_round_trip():
         assert np.all(err <= np.maximum(np.abs(a) * 2.0 ** -4, blk * 2.0 ** -9) * 1.0000001)
 
 
+def test_e2m1_decode_matches_ml_dtypes_for_all_codes():
+    import ml_dtypes
+    codes = np.arange(16, dtype=np.uint8)
+    lib = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(oracle.decode_e2m1(codes), lib)
+    assert oracle.decode_e2m1(np.uint8(0x7)) == 6.0 and oracle.decode_e2m1(np.uint8(0x1)) == 0.5
+    # only the low nibble is a code
+    assert np.array_equal(oracle.decode_e2m1(codes | 0xF0), lib)
+
+
+def test_e8m0_decode_matches_ml_dtypes_for_all_codes():
+    import ml_dtypes
+    codes = np.arange(256, dtype=np.uint8)
+    lib = codes.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    ours = oracle.decode_e8m0(codes)
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    assert np.array_equal(ours[ok], lib[ok])
+    assert oracle.decode_e8m0(np.uint8(127)) == 1.0
+
+
+def test_fp4_packing_order():
+    """Byte j of a packed row holds element 2j in its low nibble: 0x72 is (1.0, 6.0)."""
+    packed = np.array([[0x72, 0x0B]], np.uint8)
+    assert np.array_equal(oracle.unpack_fp4(packed), [[2, 7, 11, 0]])
+    vals = oracle.dequantize_mxfp4(np.tile(packed, (1, 8)), np.array([[128]], np.uint8))
+    assert np.array_equal(vals[0, :4], [2.0, 12.0, -3.0, 0.0])
+
+
+def test_mxfp4_round_trip():
+    rng = np.random.default_rng(4)
+    # rows and 32-element blocks of very different magnitudes so a misplaced scale shows
+    a = (rng.standard_normal((64, 256)) * np.exp2(rng.integers(-6, 6, (64, 8))).repeat(32, 1)
+         ).astype(np.float32)
+    a[3, 32:64] = 0.0
+    packed, sc = inputs.to_mxfp4(a)
+    back = oracle.dequantize_mxfp4(packed.numpy(), sc.numpy())
+    s = np.exp2(sc.numpy().astype(np.float64) - 127.0).repeat(32, 1)
+    # nearest of E2M1's values (steps of 0.5 below 2, 1 below 4, 2 below 6, relative to s):
+    # at most half a step away
+    assert np.all(np.abs(back - a) <= np.maximum(np.abs(a) * 2.0 ** -2, s * 2.0 ** -2) * 1.0000001)
+    assert np.all(np.abs(a) <= 6.0 * s)
+    assert np.all(back[3, 32:64] == 0.0)
+
+
+def test_table_mxfp4_helper_equals_oracle():
+    from helpers import dequant_mxfp4_fast
+    rng = np.random.default_rng(6)
+    packed = rng.integers(0, 256, (64, 128)).astype(np.uint8)
+    packed[0, :] = np.arange(128) * 2
+    packed[1, :] = np.arange(128) * 2 + 1
+    sc = rng.integers(100, 150, (64, 8)).astype(np.uint8)
+    assert np.array_equal(dequant_mxfp4_fast(packed, sc), oracle.dequantize_mxfp4(packed, sc))
+
+
+def test_table_dequant_helper_equals_oracle():
+    """The tests' table-driven block dequantisation (used on whole expert weight sets) gives
+    oracle.dequantize_blocks's values bit for bit, every code and block shape included."""
+    from helpers import dequant_fast
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, (256, 384)).astype(np.uint8)
+    codes[0, :256] = np.arange(256)
+    for br, bc in ((1, 128), (128, 128)):
+        s = np.exp2(rng.integers(-10, 10, (256 // br, 384 // bc))).astype(np.float32)
+        a = dequant_fast(codes, s, br, bc)
+        b = oracle.dequantize_blocks(codes, s, br, bc)
+        assert np.array_equal(np.isnan(a), np.isnan(b))
+        assert np.array_equal(a[~np.isnan(a)], b[~np.isnan(b)])
+
+
 def test_softmax_k_equals_E_is_full_softmax():
     rng = np.random.default_rng(0)
     L = rng.uniform(-3, 3, (32, 7))
