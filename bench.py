@@ -51,6 +51,10 @@ def parse():
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling case: the workload with only this many routed experts "
                          "(drawn without the stored recipe; not a bench line)")
+    ap.add_argument("--stages-only", action="store_true",
+                    help="time moe_route, moe_permute and moe_combine alone at the workload's "
+                         "sizes on random inputs (no expert weights; profiling case, not a "
+                         "bench line)")
     ap.add_argument("--fp8-peak", action="store_true",
                     help="measure the dense e4m3 GEMM peak (cuBLASLt) on cuda:0, print it, exit")
     return ap.parse_args()
@@ -317,8 +321,9 @@ def _weight_values(w, s):
     import torch
     if s is None:
         return w.double().numpy()
-    if s.dtype == torch.uint8:           # MXFP4: packed E2M1 codes + E8M0 scale codes
-        return oracle.dequantize_mxfp4(w.numpy(), s.numpy())
+    if s.dtype == torch.uint8:           # MXFP4: packed E2M1 codes + E8M0 scale atoms
+        from sparse_expert_moe_b200 import inputs
+        return oracle.dequantize_mxfp4(w.numpy(), inputs.scale_rows(s.numpy()).numpy())
     return oracle.dequantize_blocks(w.view(torch.uint8).numpy(), s.numpy(), 128, 128)
 
 
@@ -358,10 +363,14 @@ def time_oracle(light, rows, stored):
 
     t0 = time.perf_counter()
     xv = _act_values(light, rows)
+    expert_x = None
+    if spec.act == "bf16" and spec.weight in ("e4m3", "e2m1"):   # quantised in the permutation
+        codes, sc = oracle.quantize_e4m3_blocks(xv)
+        expert_x = oracle.dequantize_blocks(codes, sc, 1, 128)
     oracle.layer_forward(xv, light["wr"].double().numpy(), spec.score, spec.top_k,
                          lambda e: expert("r", e), spec.E,
                          [(lambda s=s: expert("s", s)) for s in range(spec.n_shared)],
-                         sel_bias=light["bias"])
+                         sel_bias=light["bias"], expert_x=expert_x)
     return time.perf_counter() - t0
 
 
@@ -534,6 +543,27 @@ def decode_uniform(moe, inputs, layer, wl, y, idx, gw, K, W, stream, dev, barrie
             "stages_ms": stage_ms}
 
 
+def time_graph(moe, layer, x, xs, y, idx, gw, K, W, stream, dev, barrier, max_over_ranks):
+    """K replays of the layer recorded once as a CUDA graph (moe_layer_graph_*), device time
+    between a barrier + synchronize on both sides: ms per step (max over ranks)."""
+    import torch
+    g = moe.LayerGraph(layer.cfg, layer.weights, x, xs, y, idx, gw, layer.ws)
+    for _ in range(W):
+        g.launch(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K):
+        g.launch(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    g.close()
+    return max_over_ranks(e0.elapsed_time(e1)) / K
+
+
 def launches_per_step(spec):
     """Kernels one ``moe_layer_forward`` launches: router GEMM, route, permute (count and
     gather for T <= 256, else count, rank and gather), plan, FFN1, FFN2, combine; the
@@ -608,6 +638,10 @@ def run_ours(args):
 
     # end to end through the public call, pipelined as a serving loop runs it
     e2e_ms, h2d, d2h = time_e2e(layer, wl, y, idx, gw, stream, K, dev, barrier, max_over_ranks)
+    graph_ms = None
+    if spec.T <= 256:      # decode-sized batches: the layer's launches as one graph
+        graph_ms = time_graph(moe, layer, x, xs, y, idx, gw, K, args.warmup, stream, dev, barrier,
+                              max_over_ranks)
     idx_np = idx.cpu().numpy()
     peaks, peak_src = load_peaks()
     uniform = None
@@ -688,6 +722,10 @@ def run_ours(args):
     }
     if uniform is not None:
         line["decode_uniform"] = uniform
+    if graph_ms is not None:
+        line["graph"] = {"ms_per_step": graph_ms, "value": spec.T * world / (graph_ms * 1e-3),
+                         "unit": "tokens/s",
+                         "how": "moe_layer_graph_launch: the layer recorded once as a CUDA graph"}
     if not args.no_cpu_baseline and world == 1:
         host = {n: getattr(wl, n) for n in ("w13", "w2", "ws13", "ws2", "w13_s", "w2_s", "ws13_s",
                                             "ws2_s")}
@@ -699,8 +737,76 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_stages(args):
+    """moe_route, moe_permute and moe_combine alone at the sizes of a workload, on random
+    inputs of its shapes and dtypes (the bandwidth-bound stages around the expert GEMMs),
+    each timed over K calls with CUDA events, an L2 flush (a 256 MB write) before every
+    call; GB/s against the algorithmic bytes of ``small_stage_bytes``."""
+    import torch
+    from sparse_expert_moe_b200 import inputs, moe
+    spec = inputs.SPECS[args.workload]
+    if args.tokens:
+        from dataclasses import replace
+        spec = replace(spec, T=args.tokens)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, d, E, k, S = spec.T, spec.d_model, spec.E, spec.top_k, spec.n_shared
+    R = T * k
+    g = torch.Generator(device=dev).manual_seed(0)
+    cfg = moe.config_from_spec(spec)
+    logits = torch.randn((T, E), generator=g, device=dev)
+    bias = None if spec.score != "sigmoid_bias" else 0.1 * torch.rand(E, generator=g, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gw = torch.empty((T, k), dtype=torch.float32, device=dev)
+    fp8 = spec.act == "e4m3"
+    x = torch.randn((T, d), generator=g, device=dev).to(torch.bfloat16)
+    xs = xps = None
+    if fp8:
+        x = x.to(torch.float8_e4m3fn).view(torch.uint8)
+        xs = torch.ones((T, d // 128), device=dev)
+        xps = torch.empty((R, d // 128), device=dev)
+    x_perm = torch.empty((R, d), dtype=x.dtype, device=dev)
+    perm_token = torch.empty(R, dtype=torch.int32, device=dev)
+    inv_perm = torch.empty((T, k), dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    y_perm = torch.randn((R, d), generator=g, device=dev).to(torch.bfloat16)
+    y_sh = torch.randn((S, T, d), generator=g, device=dev).to(torch.bfloat16) if S else None
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = {
+        "route": lambda: moe.moe_route(cfg, logits, bias, idx, gw),
+        "permute": lambda: moe.moe_permute(cfg, idx, x, xs, x_perm, xps, perm_token, inv_perm,
+                                           offsets, ws),
+        "combine": lambda: moe.moe_combine(cfg, y_perm, inv_perm, gw, y_sh, y),
+    }
+    nbytes = small_stage_bytes(spec)
+    out = {}
+    for name, fn in calls.items():
+        for _ in range(args.warmup):
+            fn()
+        ms = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        t = statistics.median(ms)
+        gbs = nbytes[name] / (t * 1e-3) / 1e9
+        out[name] = {"ms": t, "bytes": nbytes[name], "gbs": gbs, "frac": gbs / load_peaks()[0]["hbm_gbs"]}
+    status = moe.moe_read_device_status(ws)
+    print(json.dumps({"workload": args.workload, "T": T, "stages": out, "device_status": status,
+                      "how": "median of --steps calls, L2 flushed before each"}), flush=True)
+
+
 def main():
     args = parse()
+    if args.stages_only:
+        run_stages(args)
+        return
     if args.fp8_peak:
         print(json.dumps(measure_fp8_peak("cuda:0")), flush=True)
         return

@@ -37,10 +37,13 @@
  *  - dtypes: activations MOE_BF16, MOE_E4M3 (with fp32 1x128 scales) or
  *    MOE_F32; weights the same family (bf16 weights with bf16 activations,
  *    e4m3 weights + fp32 128x128 block scales with e4m3 activations, f32 with
- *    f32), or MOE_E2M1 (MXFP4) weights with MOE_E4M3 activations.  f32 inputs
- *    are rounded to bf16 (nearest even) on entry; the tensor cores compute in
- *    bf16 (or e4m3 / e2m1 x e4m3) with fp32 accumulation.  The router weights
- *    are bf16 for the bf16, e4m3 and e2m1 families, f32 for f32.
+ *    f32), or MOE_E2M1 (MXFP4) weights with MOE_E4M3 activations; or MOE_BF16
+ *    activations with MOE_E4M3 or MOE_E2M1 weights, quantised to e4m3 in the
+ *    permutation (see moe_permute).  f32 inputs are rounded to bf16 (nearest
+ *    even) on entry; the tensor cores compute in bf16 (or e4m3 / e2m1 x e4m3)
+ *    with fp32 accumulation.  The router weights are bf16 for the bf16, e4m3 and
+ *    e2m1 families, f32 for f32; the router takes x as given (bf16, or e4m3
+ *    dequantised exactly).
  *    FP8 block scales must be positive normal powers of two (exactly what the
  *    tensor cores' UE8M0 scale factors represent); any other scale sets the
  *    device status MOE_ERR_DEVICE_VALUE.  MXFP4 scale bytes are used as given
@@ -90,7 +93,11 @@ typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_BIAS = 1 } moe_score_fn;
 
 /* MOE_E2M1: FP4 weights in the OCP MXFP4 format -- E2M1 codes packed two per byte (element
  * 2j in the low nibble of byte j), one E8M0 scale byte (2^(code - 127)) per 32 consecutive
- * elements along K -- taken with e4m3 activations ("FP8/FP4 grouped GEMM", GC-MoE title). */
+ * elements along K -- taken with e4m3 activations ("FP8/FP4 grouped GEMM", GC-MoE title).
+ * The scale bytes of a [rows, K] weight matrix are stored as 512-byte atoms, one per 128
+ * rows x 128 K-elements, [rows/128][K/128][512]: inside an atom the scale of row r (0..127)
+ * and 32-element run q (0..3) sits at byte (r % 32) * 16 + (r / 32) * 4 + q -- the layout
+ * the tensor cores' scale-factor copy takes, so the kernels copy atoms without reshuffling. */
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2, MOE_E2M1 = 3 } moe_dtype;
 
 /* The layer's sizes: T tokens x d_model activations, E routed experts, top_k,
@@ -109,9 +116,10 @@ typedef struct {
  *   w2     [E, d, I]       per expert down projection
  *   w13_s, w2_s            block scales of the weights:
  *                          e4m3: fp32 [E, 2I/128, d/128] and [E, d/128, I/128];
- *                          e2m1: uint8 E8M0 codes [E, 2I, d/32] and [E, d, I/32]
- *                          (w13 is then [E, 2I, d/2] bytes, w2 [E, d, I/2]; both
- *                          32-byte aligned); unused (NULL) otherwise
+ *                          e2m1: uint8 E8M0 codes in scale atoms (see MOE_E2M1),
+ *                          [E, 2I/128, d/128, 512] and [E, d/128, I/128, 512],
+ *                          16-byte aligned (w13 is then [E, 2I, d/2] bytes, w2
+ *                          [E, d, I/2], both 32-byte aligned); unused (NULL) otherwise
  *   ws13 [S, 2I, d], ws2 [S, d, I] (+ ws13_s, ws2_s): shared experts (NULL when S = 0) */
 typedef struct {
   const void *wr;
@@ -146,7 +154,14 @@ MOE_API moe_status moe_route(const moe_config *cfg, const float *logits, const f
  *   perm_token    [T*k] int32  token of each permuted row (output)
  *   inv_perm      [T, k] int32 permuted row of (token, slot) (output)
  *   group_offsets [E+1] int32  exclusive prefix of group sizes (output)
- *   ws, ws_bytes  workspace (>= moe_workspace_size) */
+ *   ws, ws_bytes  workspace (>= moe_workspace_size)
+ * Quantise-in-permute: with bf16 activations and e4m3 or FP4 expert weights
+ * (cfg->act MOE_BF16, cfg->weight MOE_E4M3 / MOE_E2M1) the rows are quantised to
+ * e4m3 in the same pass, as the expert GEMMs take them: each token's 128-value
+ * block gets the scale 2^e, e the smallest integer with amax <= 448 * 2^e (e = 0
+ * for an all-zero block), and each value x becomes e4m3(x / 2^e), round to nearest
+ * even.  x_perm [T*k, d] then receives e4m3 codes and x_perm_scale [T*k, d/128]
+ * (required) the fp32 scales 2^e; x_scale is unused. */
 MOE_API moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, const void *x,
                        const float *x_scale, void *x_perm, float *x_perm_scale,
                        int32_t *perm_token, int32_t *inv_perm, int32_t *group_offsets,
@@ -158,6 +173,8 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, c
  * where cudaMalloc (which may synchronise the device) is not allowed.  The pages
  * have no counterpart: it is the same permutation with the same arguments and
  * results as moe_permute, minus ws / ws_bytes.
+ * bf16 rows for e4m3 or FP4 experts (the quantising permutation) are not taken
+ * here: MOE_ERR_UNSUPPORTED.
  * Its scratch is a fixed array inside the library (about 1 MiB per GPU that
  * loads the library, held until the process exits), so it accepts only
  * ceil(T / 256) * E <= 262144 (for example T <= 65536 with E <= 1024); larger
@@ -194,8 +211,10 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *top
  *   n_rows          rows allocated in a and y (>= offsets[G], <= T*k + n_shared*T,
  *                   the most the workspace holds); nothing past row n_rows is
  *                   read or written
- *   a               [offsets[G], d] rows (cfg->act); a_scale [rows, d/128] fp32
- *                   for e4m3, else NULL.  For the f32 family a, w13 and w2 are
+ *   a               [offsets[G], d] rows in the token dtype of the expert GEMMs:
+ *                   cfg->act, except e4m3 whenever the weights are e4m3 or FP4
+ *                   (as moe_permute returns them); a_scale [rows, d/128] fp32 for
+ *                   e4m3 rows, else NULL.  For the f32 family a, w13 and w2 are
  *                   rounded to bf16 into the workspace first.
  *   w13, w2         [G, 2I, d], [G, d, I] (+ block scales for e4m3 and e2m1 weights,
  *                   laid out as in moe_weights)
@@ -238,6 +257,29 @@ MOE_API moe_status moe_layer_forward_staged(const moe_config *cfg, const moe_wei
                                             int32_t *topk_idx_out, float *topk_w_out, void *ws,
                                             size_t ws_bytes, cudaStream_t stream,
                                             cudaEvent_t *stage_events);
+
+/* The whole layer recorded once into a CUDA graph and replayed: every kernel of
+ * moe_layer_forward (8 to 14 launches) goes to the GPU as one graph launch, which
+ * removes the per-launch host cost and the gaps between the layer's kernels on a
+ * decode step ("Fused single-kernel decode layer ... or a CUDA-graph capture"; the
+ * 3-node CUDA graph of the GC-MoE key changes).
+ *  moe_layer_graph_create  checks its arguments as moe_layer_forward does, then
+ *      records the layer for exactly these pointers and sizes on an internal stream
+ *      (no kernel runs) and instantiates the graph into *graph_out.  The graph reads x
+ *      (and x_scale) and writes y, the routing outputs and ws at the addresses given
+ *      here: to run the layer on new activations, write them into x and launch again.
+ *      It allocates host memory for the handle and the graph; no device memory.
+ *  moe_layer_graph_launch  enqueues one layer call on `stream` (stream-ordered, like
+ *      moe_layer_forward).  Launches of one graph must not overlap on the GPU: they
+ *      share the workspace.
+ *  moe_layer_graph_destroy frees the handle (after its launches have completed). */
+typedef struct moe_layer_graph_t *moe_layer_graph;
+MOE_API moe_status moe_layer_graph_create(const moe_config *cfg, const moe_weights *weights,
+                                          const void *x, const float *x_scale, void *y,
+                                          int32_t *topk_idx_out, float *topk_w_out, void *ws,
+                                          size_t ws_bytes, moe_layer_graph *graph_out);
+MOE_API moe_status moe_layer_graph_launch(moe_layer_graph graph, cudaStream_t stream);
+MOE_API moe_status moe_layer_graph_destroy(moe_layer_graph graph);
 
 /* Self-test of the device-side failure path (no counterpart on the pages): a
  * tiny kernel waits on a barrier that nothing completes, gives up after

@@ -134,6 +134,37 @@ def dequantize_mxfp4(packed, scale_codes, block: int = 32) -> np.ndarray:
     return v * np.repeat(s, block, axis=-1)[..., : v.shape[-1]]
 
 
+def quantize_e4m3_blocks(x, block: int = 128):
+    """Quantise rows to e4m3 with one power-of-two scale per `block` consecutive values of a
+    row (the activation quantisation of the FP8 path; GC-MoE key change on fused
+    requantisation).  Reading: the scale of a block is 2^e for the smallest integer e with
+    amax <= 448 * 2^e (448 = the largest e4m3 magnitude; e = 0 for an all-zero block;
+    e kept within the E8M0 range [-127, 127]); each value x / 2^e (exact: a power-of-two
+    division) goes to the nearest e4m3 value, ties to the even code, with its sign (a
+    negative value that rounds to zero gives negative zero).
+
+    Returns (codes uint8 [R, C], scales fp64 [R, C / block])."""
+    x = np.asarray(x, np.float64)
+    R, C = x.shape
+    amax = np.abs(x).reshape(R, C // block, block).max(axis=2)
+    m, e = np.frexp(amax / 448.0)                   # amax / 448 = m * 2^e, m in [0.5, 1)
+    e = np.where(m == 0.5, e - 1, e)                 # exact powers of two
+    e = np.where(amax > 0, e, 0)
+    e = np.clip(e, -127, 127)
+    scales = np.exp2(e.astype(np.float64))
+    q = x / np.repeat(scales, block, axis=1)
+    # the non-negative finite e4m3 values in code order 0x00 .. 0x7E (increasing)
+    values = decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    a = np.abs(q)
+    hi = np.clip(np.searchsorted(values, a, side="left"), 0, 0x7E)   # values[hi] >= a
+    lo = np.clip(hi - 1, 0, 0x7E)
+    d_lo, d_hi = a - values[lo], values[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(np.signbit(q), code | 0x80, code).astype(np.uint8)
+    return code, scales
+
+
 # ---------------------------------------------------------------------------
 # Router: gate(x), scores, top-k, gates
 # ---------------------------------------------------------------------------
@@ -273,10 +304,13 @@ def combine(y_perm, inv_perm, gates, y_shared=None) -> np.ndarray:
 
 
 def layer_forward(x, wr, score: str, k: int, expert_weights, n_experts: int,
-                  shared_weights=(), sel_bias=None, return_routing: bool = False):
+                  shared_weights=(), sel_bias=None, return_routing: bool = False,
+                  expert_x=None):
     """The whole layer, step by step.
 
     x               [T, d] activation values (already decoded to real numbers)
+    expert_x        [T, d] the values the experts (routed and shared) take instead of x,
+                    e.g. x quantised for FP8 expert weights; the router always takes x
     wr              [E, d] router weights
     expert_weights  callable e -> (w13 [2I, d], w2 [d, I]); called once per
                     expert that has at least one row, so only one expert's
@@ -287,6 +321,8 @@ def layer_forward(x, wr, score: str, k: int, expert_weights, n_experts: int,
     logits = router_logits(x, wr)
     idx, gates = route(logits, score, k, sel_bias)
     offsets, perm_token, inv_perm = permute(idx, n_experts)
+    if expert_x is not None:
+        x = np.asarray(expert_x, np.float64)
     x_perm = x[perm_token]
     d = x.shape[1]
     y_perm = np.zeros((x_perm.shape[0], d), np.float64)

@@ -22,6 +22,13 @@ constexpr int kHdrNGroups = 3;
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
+// The expert GEMMs take e4m3 token rows: e4m3 activations, or bf16 activations quantised
+// in the permutation because the expert weights are e4m3 or FP4.
+inline bool tok_e4m3(const moe_config& c) {
+  return c.act == MOE_E4M3 || c.weight == MOE_E4M3 || c.weight == MOE_E2M1;
+}
+inline bool quant_in_permute(const moe_config& c) { return c.act == MOE_BF16 && tok_e4m3(c); }
+
 // Byte offsets of every workspace region for one configuration.
 struct Layout {
   size_t logits, topk_idx, topk_w, offsets, chunk_counts, perm_token, inv_perm, x_perm, chunks,
@@ -36,7 +43,8 @@ struct Layout {
     rows_all = R + S * T;
     n_chunk_max = max_chunks(rows_all, E + S);
     const bool f32 = c.act == MOE_F32;
-    const bool fp8 = c.act == MOE_E4M3;            // e4m3 activations (e4m3 or FP4 weights)
+    const bool fp8 = tok_e4m3(c);                  // e4m3 token operand (e4m3 or FP4 weights)
+    const bool q8 = fp8 && c.act == MOE_BF16;      // bf16 activations quantised in the permute
     const bool w8 = c.weight == MOE_E4M3;          // fp32 block scales re-encoded per call
     size_t o = kHeaderBytes;
     auto take = [&](size_t bytes) {
@@ -56,7 +64,8 @@ struct Layout {
     grp_cp = take(sizeof(int32_t) * 2 * (E + S + 1));
     h = take(2 * rows_all * I);
     y_rows = take(2 * rows_all * d);
-    x_bf16 = take(f32 || fp8 ? 2 * T * d : 0);
+    x_bf16 = take(f32 || fp8 ? 2 * T * d : 0);   // q8: the quantised x [T, d] e4m3
+    (void)q8;
     wr_bf16 = take(f32 ? 2 * E * d : 0);
     w13_bf16 = take(f32 ? 2 * (E + S) * 2 * I * d : 0);
     w2_bf16 = take(f32 ? 2 * (E + S) * d * I : 0);
@@ -80,10 +89,7 @@ inline int* status_word(void* ws) { return at<int>(ws, kHdrStatus * sizeof(int))
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
-// bytes of a weight row of `k` elements
-inline int64_t weight_row_bytes(const moe_config& c, int64_t k) {
-  return c.weight == MOE_E2M1 ? k / 2 : (c.weight == MOE_E4M3 ? k : (c.weight == MOE_F32 ? 4 * k : 2 * k));
-}
+
 
 moe_status check_config(const moe_config* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -101,7 +107,9 @@ moe_status check_config(const moe_config* c) {
   const bool fam_f32 = c->act == MOE_F32 && c->weight == MOE_F32;
   const bool fam_fp8 = c->act == MOE_E4M3 && c->weight == MOE_E4M3;
   const bool fam_w4a8 = c->act == MOE_E4M3 && c->weight == MOE_E2M1;
-  if (!(fam_bf16 || fam_f32 || fam_fp8 || fam_w4a8)) return MOE_ERR_UNSUPPORTED;
+  // bf16 activations into e4m3 or FP4 experts: quantised to e4m3 in the permutation
+  const bool fam_q8 = c->act == MOE_BF16 && (c->weight == MOE_E4M3 || c->weight == MOE_E2M1);
+  if (!(fam_bf16 || fam_f32 || fam_fp8 || fam_w4a8 || fam_q8)) return MOE_ERR_UNSUPPORTED;
   if (c->out != MOE_BF16 && c->out != MOE_F32) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -208,8 +216,7 @@ void copy_maps(CUtensorMap (&dst)[4], const CUtensorMap (&src)[4]) {
 // One segment of the FP8 block-scaled expert GEMMs: token rows `a` (e4m3) with their
 // UE8M0 scale factors a_sf [d/128][a_rows], and `groups` experts' weights -- e4m3 with
 // UE8M0 block scale factors wsf13 / wsf2 (re-encoded from the caller's fp32 128x128
-// scales), or FP4 (packed E2M1) with the caller's E8M0 codes wsc13 [rows][d/32] /
-// wsc2 [rows][I/32].
+// scales), or FP4 (packed E2M1) with the caller's E8M0 scale atoms wsc13 / wsc2.
 struct Fp8Seg {
   const void* a;
   const uint32_t* a_sf;
@@ -218,9 +225,10 @@ struct Fp8Seg {
   const void* w2;
   const uint4* wsf13;
   const uint4* wsf2;
-  const uint8_t* wsc13;
-  const uint8_t* wsc2;
+  const uint4* wsc13;
+  const uint4* wsc2;
   int64_t groups;
+  const int32_t* gidx;   // gather-on-load: token row n of a chunk is row gidx[b_row + n] of a
 };
 
 bool weight_map(CUtensorMap* m, const void* w, int64_t rows, int64_t cols, bool w4) {
@@ -232,7 +240,7 @@ bool weight_map(CUtensorMap* m, const void* w, int64_t rows, int64_t cols, bool 
 // (e4m3) and its scales live in the workspace; y has rows_all rows.
 moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8Seg& s0,
                        const Fp8Seg& s1, int64_t rows_all, void* y, int chunk_rows, cudaStream_t s,
-                       cudaEvent_t* ev = nullptr) {
+                       cudaEvent_t* ev = nullptr, bool gather = false) {
   const int64_t d = c.d_model, I = c.d_ff;
   const bool w4 = c.weight == MOE_E2M1;
   void* h = at<void>(ws, L.h);
@@ -251,6 +259,13 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8
   g.mode = w4 ? kFFN1F4 : kFFN1F8;
   g.halves = chunk_rows == 2 * kChunkRowsFP8;
   g.tile_tokens = chunk_rows == kChunkRowsNarrow ? kChunkRowsNarrow : kChunkRows;
+  // gather-on-load: token rows straight from the (unpermuted) e4m3 activations
+  g.gather = gather && chunk_rows != kChunkRowsNarrow;
+  for (int i = 0; i < 2; ++i) {
+    g.gsrc[i] = seg[i]->a;
+    g.gidx[i] = seg[i]->gidx;
+  }
+  g.g_ld = static_cast<int>(d);
   for (int i = 0; i < 2; ++i) {
     const Fp8Seg& q = *seg[i];
     if (!weight_map(&g.wmap[i], q.w13, q.groups * 2 * I, d, w4) ||
@@ -262,7 +277,6 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8
     g.tsf_ld[i] = static_cast<int>(q.a_rows);
     g.tsf_rows[i] = static_cast<int>(q.a_rows);
   }
-  g.wsc_ld = static_cast<int>(d / 32);
   g.n_mblk = static_cast<int>(I / 128);
   g.k_blocks = static_cast<int>(d / 128);
   g.w_rows_per_group = static_cast<int>(2 * I);
@@ -277,8 +291,10 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
+  const bool m256 = false;
   g.mode = w4 ? kFFN2F4 : kFFN2F8;
   g.halves = false;
+  g.gather = false;
   g.tile_tokens = chunk_rows;
   if (!make_tok_maps(g.tmap[0], h, rows_all, I, true)) return MOE_ERR_CUDA;
   copy_maps(g.tmap[1], g.tmap[0]);
@@ -291,8 +307,7 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8
     g.tsf_ld[i] = static_cast<int>(rows_all);
     g.tsf_rows[i] = static_cast<int>(rows_all);
   }
-  g.wsc_ld = static_cast<int>(I / 32);
-  g.n_mblk = static_cast<int>(d / 128);
+  g.n_mblk = static_cast<int>(m256 ? d / 256 : d / 128);
   g.k_blocks = static_cast<int>(I / 128);
   g.w_rows_per_group = static_cast<int>(d);
   g.wsf_rb_per_group = static_cast<int>(d / 128);
@@ -354,6 +369,7 @@ moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
+  g.gather = false;
   const bool m512 = d % 512 == 0 && chunk_rows == kChunkRowsNarrow;
   const bool m256 = d % 256 == 0 && !m512;
   g.mode = m512 ? kFFN2M512 : (m256 ? kFFN2M256 : kFFN2);
@@ -419,6 +435,13 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
   const Layout L(*cfg);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (quant_in_permute(*cfg)) {   // bf16 rows -> e4m3 rows + fp32 power-of-two scales
+    if (cfg->T > 0 && !x_perm_scale) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_permute_quant(
+        topk_idx, cfg->T, cfg->E, cfg->top_k, x, cfg->d_model, x_perm, x_perm_scale, nullptr,
+        nullptr, nullptr, perm_token, inv_perm, group_offsets, at<int32_t>(ws, L.chunk_counts),
+        at<unsigned>(ws, kHdrPermuteDone * sizeof(int)), status_word(ws), stream));
+  }
   const bool fp8 = cfg->act == MOE_E4M3;
   if (fp8 && cfg->T > 0 && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
   const int elem = cfg->act == MOE_F32 ? 4 : (fp8 ? 1 : 2);
@@ -439,8 +462,11 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
   if (n_groups <= 0 || n_groups > 1024 || n_rows < 0) return MOE_ERR_INVALID_ARG;
   if (!group_offsets || !a || !w13 || !w2 || !y || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(w13) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
-  // packed FP4 weights are loaded by TMA from 32-byte aligned bases
-  if (cfg->weight == MOE_E2M1 && (!aligned32(w13) || !aligned32(w2))) return MOE_ERR_INVALID_ARG;
+  // packed FP4 weights are loaded by TMA from 32-byte aligned bases, their scale atoms in
+  // 16-byte copies
+  if (cfg->weight == MOE_E2M1 && (!aligned32(w13) || !aligned32(w2) || !aligned16(w13_s) ||
+                                  !aligned16(w2_s)))
+    return MOE_ERR_INVALID_ARG;
   const Layout L(*cfg);
   if (n_rows > L.rows_all) return MOE_ERR_UNSUPPORTED;
   // the workspace's chunk list and group tables are sized for E + n_shared groups
@@ -465,16 +491,16 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
     w13_b = at<void>(ws, L.w13_bf16);
     w2_b = at<void>(ws, L.w2_bf16);
   }
-  if (cfg->act == MOE_E4M3) {
+  if (tok_e4m3(*cfg)) {   // e4m3 token rows (as moe_permute gives them for e4m3 / FP4 experts)
     if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
     const bool w4 = cfg->weight == MOE_E2M1;
     uint32_t* a_sf = at<uint32_t>(ws, L.a_sf);
-    Fp8Seg s0{a, a_sf, n_rows, w13, w2, nullptr, nullptr, nullptr, nullptr, n_groups};
+    Fp8Seg s0{a, a_sf, n_rows, w13, w2, nullptr, nullptr, nullptr, nullptr, n_groups, nullptr};
     st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(a), a_scale, n_rows,
                                          static_cast<int>(d), nullptr, a_sf, status_word(ws), stream));
     if (w4) {
-      s0.wsc13 = static_cast<const uint8_t*>(w13_s);
-      s0.wsc2 = static_cast<const uint8_t*>(w2_s);
+      s0.wsc13 = static_cast<const uint4*>(w13_s);
+      s0.wsc2 = static_cast<const uint4*>(w2_s);
     } else {
       s0.wsf13 = at<uint4>(ws, L.wsf13);
       s0.wsf2 = at<uint4>(ws, L.wsf2);
@@ -542,14 +568,17 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if (!aligned16(x) || !aligned16(y) || !aligned16(wts->wr) || !aligned16(wts->w13) ||
       !aligned16(wts->w2) || !aligned16(wts->ws13) || !aligned16(wts->ws2))
     return MOE_ERR_INVALID_ARG;
-  const bool fp8 = c.act == MOE_E4M3;
+  const bool fp8 = tok_e4m3(c);            // e4m3 token operand of the expert GEMMs
+  const bool q8 = quant_in_permute(c);     // ... quantised from bf16 x in the permutation
   const bool w4 = c.weight == MOE_E2M1;
-  if (fp8 && (!x_scale || !wts->w13_s || !wts->w2_s ||
+  if (fp8 && ((!q8 && !x_scale) || !wts->w13_s || !wts->w2_s ||
               (c.n_shared > 0 && (!wts->ws13_s || !wts->ws2_s))))
     return MOE_ERR_INVALID_ARG;
-  // packed FP4 weights are loaded by TMA from 32-byte aligned bases
+  // packed FP4 weights are loaded by TMA from 32-byte aligned bases, their scale atoms in
+  // 16-byte copies
   if (w4 && (!aligned32(wts->w13) || !aligned32(wts->w2) || !aligned32(wts->ws13) ||
-             !aligned32(wts->ws2)))
+             !aligned32(wts->ws2) || !aligned16(wts->w13_s) || !aligned16(wts->w2_s) ||
+             !aligned16(wts->ws13_s) || !aligned16(wts->ws2_s)))
     return MOE_ERR_INVALID_ARG;
   const Layout L(c);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -594,8 +623,10 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
   const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
   if (fp8) {
-    st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(x), x_scale, c.T,
-                                         static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf, status, s));
+    if (!q8)
+      st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(x), x_scale, c.T,
+                                           static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf,
+                                           status, s));
     if (!w4) {   // e4m3 weights: fp32 block scales -> UE8M0 scale factors
       auto wsf = [&](const void* src, size_t n, uint4* dst) {
         return cuda_status(launch_weight_sf(static_cast<const float*>(src), n, dst, status, s));
@@ -606,7 +637,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
       if (st == MOE_OK && S > 0) st = wsf(wts->ws2_s, S * n2, wsf2 + E * n2);
     }
     if (st != MOE_OK) return st;
-    x_router = at<void>(ws, L.x_bf16);
+    if (!q8) x_router = at<void>(ws, L.x_bf16);    // e4m3 x dequantised for the router
   }
 
   // 1. router GEMM: logits[T, E] = x Wr^T (fp32)
@@ -643,25 +674,46 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if (st != MOE_OK) return st;
   if ((st = mark(2)) != MOE_OK) return st;
 
-  // 3. permute (bf16 rows, or e4m3 rows + their scale factors)
+  // 3. permute.  Groups hold at most T rows, which picks the token-tile width of the expert
+  // GEMMs.  With e4m3 token rows on wide tiles (more than 128 tokens) the first GEMM gathers
+  // its token rows from x itself (gather-on-load), so only the routing tables are built
+  // here; otherwise the rows are copied into x_perm (bf16 rows, or e4m3 rows + scale
+  // factors).  bf16 rows keep the copy: measured on the R1 prefill layer, the first GEMM
+  // fed by TMA from x_perm is faster than with gathered rows by more than the copy costs.
+  const int chunk_rows = fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T);
+  const bool gather = fp8 && chunk_rows != kChunkRowsNarrow;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm_token = at<int32_t>(ws, L.perm_token);
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   void* x_perm = at<void>(ws, L.x_perm);
   uint32_t* x_perm_sf = at<uint32_t>(ws, L.x_perm_sf);
-  st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(fp8 ? d : d * 2),
-                                  nullptr, 0, x_perm, nullptr, perm_token, inv_perm, offsets,
-                                  at<int32_t>(ws, L.chunk_counts),
-                                  at<unsigned>(ws, kHdrPermuteDone * sizeof(int)), status, s));
-  if (st == MOE_OK && fp8)
-    st = cuda_status(launch_gather_sf(x_sf, c.T, static_cast<int>(d / 128), perm_token, offsets + E,
-                                      static_cast<int>(R), x_perm_sf, s));
+  int32_t* counts = at<int32_t>(ws, L.chunk_counts);
+  unsigned* ticket = at<unsigned>(ws, kHdrPermuteDone * sizeof(int));
+  const void* x_tok = x_b;     // the unpermuted token rows the expert GEMMs take
+  if (q8) {
+    // bf16 rows quantised to e4m3 in the copy: every token's own quantised row (the shared
+    // experts' rows and, with gather-on-load, the routed ones) and, on decode-sized tiles,
+    // x_perm with its UE8M0 scale words
+    st = cuda_status(launch_permute_quant(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(d),
+                                          gather ? nullptr : x_perm, nullptr,
+                                          gather ? nullptr : x_perm_sf, at<void>(ws, L.x_bf16), x_sf,
+                                          perm_token, inv_perm, offsets, counts, ticket, status, s));
+    x_tok = at<void>(ws, L.x_bf16);
+  } else if (gather) {
+    st = cuda_status(launch_permute_index(idx, c.T, c.E, c.top_k, perm_token, inv_perm, offsets,
+                                          counts, ticket, status, s));
+  } else {
+    st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(fp8 ? d : d * 2),
+                                    nullptr, 0, x_perm, nullptr, perm_token, inv_perm, offsets,
+                                    counts, ticket, status, s));
+    if (st == MOE_OK && fp8)
+      st = cuda_status(launch_gather_sf(x_sf, c.T, static_cast<int>(d / 128), perm_token,
+                                        offsets + E, static_cast<int>(R), x_perm_sf, s));
+  }
   if (st != MOE_OK) return st;
   if ((st = mark(3)) != MOE_OK) return st;
 
-  // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs.  Groups hold at
-  // most T rows, which picks the bf16 token-tile width.
-  const int chunk_rows = fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T);
+  // 4. plan routed groups + shared experts, 5./6. the two grouped GEMMs.
   st = cuda_status(launch_plan(offsets, c.E, static_cast<int>(R), c.n_shared, c.T,
                                static_cast<int>(R), chunk_rows,
                                at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
@@ -671,20 +723,22 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if ((st = mark(4)) != MOE_OK) return st;
   void* y_rows = at<void>(ws, L.y_rows);
   if (fp8) {
-    Fp8Seg s0{x_perm, x_perm_sf, R, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E};
-    Fp8Seg s1{x_b, x_sf, T, ws13_b, ws2_b, nullptr, nullptr, nullptr, nullptr, S};
+    Fp8Seg s0{x_perm, x_perm_sf, R, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E, nullptr};
+    if (gather) s0 = Fp8Seg{x_tok, x_sf, T, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E, perm_token};
+    Fp8Seg s1{x_tok, x_sf, T, ws13_b, ws2_b, nullptr, nullptr, nullptr, nullptr, S, nullptr};
     if (w4) {
-      s0.wsc13 = static_cast<const uint8_t*>(wts->w13_s);
-      s0.wsc2 = static_cast<const uint8_t*>(wts->w2_s);
-      s1.wsc13 = static_cast<const uint8_t*>(wts->ws13_s);
-      s1.wsc2 = static_cast<const uint8_t*>(wts->ws2_s);
+      s0.wsc13 = static_cast<const uint4*>(wts->w13_s);
+      s0.wsc2 = static_cast<const uint4*>(wts->w2_s);
+      s1.wsc13 = static_cast<const uint4*>(wts->ws13_s);
+      s1.wsc2 = static_cast<const uint4*>(wts->ws2_s);
     } else {
       s0.wsf13 = wsf13;
       s0.wsf2 = wsf2;
       s1.wsf13 = wsf13 + E * n13;
       s1.wsf2 = wsf2 + E * n2;
     }
-    st = run_ffn_fp8(c, L, ws, s0, s1, L.rows_all, y_rows, chunk_rows, s, ev ? ev + 5 : nullptr);
+    st = run_ffn_fp8(c, L, ws, s0, s1, L.rows_all, y_rows, chunk_rows, s, ev ? ev + 5 : nullptr,
+                     gather);
   } else {
     st = run_ffn(c, L, ws, x_perm, R, w13_b, w2_b, E, x_b, T, ws13_b, ws2_b, S, L.rows_all, y_rows,
                  chunk_rows, s, ev ? ev + 5 : nullptr);
@@ -729,6 +783,63 @@ moe_status moe_read_device_status(const void* ws, cudaStream_t stream, moe_statu
   if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   *out = static_cast<moe_status>(v);
   return MOE_OK;
+}
+
+}  // extern "C"
+
+struct moe_layer_graph_t {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+
+extern "C" {
+
+moe_status moe_layer_graph_create(const moe_config* cfg, const moe_weights* wts, const void* x,
+                                  const float* x_scale, void* y, int32_t* topk_idx_out,
+                                  float* topk_w_out, void* ws, size_t ws_bytes,
+                                  moe_layer_graph* graph_out) {
+  if (!graph_out) return MOE_ERR_INVALID_ARG;
+  *graph_out = nullptr;
+  // the host checks of the layer itself, before anything is recorded
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!wts || !ws) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < Layout(*cfg).total) return MOE_ERR_WORKSPACE;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+  moe_layer_graph_t* g = new moe_layer_graph_t();
+  // relaxed mode: the launch helpers set kernel attributes while recording
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    st = MOE_ERR_CUDA;
+  } else {
+    st = layer_forward_impl(cfg, wts, x, x_scale, y, topk_idx_out, topk_w_out, ws, ws_bytes, cs,
+                            nullptr);
+    const cudaError_t e = cudaStreamEndCapture(cs, &g->graph);
+    if (st == MOE_OK && e != cudaSuccess) st = MOE_ERR_CUDA;
+  }
+  if (st == MOE_OK && cudaGraphInstantiate(&g->exec, g->graph, 0) != cudaSuccess) st = MOE_ERR_CUDA;
+  cudaStreamDestroy(cs);
+  if (st != MOE_OK) {
+    moe_layer_graph_destroy(g);
+    return st;
+  }
+  *graph_out = g;
+  return MOE_OK;
+}
+
+moe_status moe_layer_graph_launch(moe_layer_graph graph, cudaStream_t stream) {
+  if (!graph || !graph->exec) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaGraphLaunch(graph->exec, stream));
+}
+
+moe_status moe_layer_graph_destroy(moe_layer_graph graph) {
+  if (!graph) return MOE_OK;
+  moe_status st = MOE_OK;
+  if (graph->exec && cudaGraphExecDestroy(graph->exec) != cudaSuccess) st = MOE_ERR_CUDA;
+  if (graph->graph && cudaGraphDestroy(graph->graph) != cudaSuccess) st = MOE_ERR_CUDA;
+  delete graph;
+  return st;
 }
 
 moe_status moe_reset_device_status(void* ws, cudaStream_t stream) {

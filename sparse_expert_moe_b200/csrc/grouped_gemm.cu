@@ -75,14 +75,19 @@ struct DevParams {
   int* status;
   // FP8 block scaling
   const uint4* wsf[2];        // [groups][row blocks][k blocks] UE8M0 x16 per 128x128 weight block
-  const uint8_t* wsc[2];      // FP4 weights: E8M0 code per row per 32 K-elements [rows][K / 32]
-  int wsc_ld;                 // K / 32
+  const uint4* wsc[2];        // FP4 weights: E8M0 codes in 512-byte scale atoms
+                              // [groups][row blocks][k blocks][32 x uint4]
   int wsf_rb_per_group;       // 128-row blocks of the weight matrix per group
   const uint32_t* tsf[2];     // [k blocks][rows] UE8M0 x4 per (128-element block, token row)
   int tsf_ld[2];
   int tsf_rows[2];
   uint32_t* out_sf;           // FFN1 (FP8): [I / 128][rows] scales of the requantised h
   int ld_out_sf;
+  // gather-on-load (first GEMM): token row n of a chunk is row gidx[b_row + n] of gsrc
+  // (gidx null: row b_row + n), g_ld bytes apart
+  const uint8_t* gsrc[2];
+  const int32_t* gidx[2];
+  int g_ld;
 };
 
 // NTW: token-tile width of the bf16 expert GEMMs.  128 by default -- half of a 256-row
@@ -91,17 +96,24 @@ struct DevParams {
 // epilogue could no longer hide behind the next tile's MMAs); 32 for decode-sized
 // batches (small token tiles leave shared memory to a deeper weight ring); 256 only for
 // the single-block FFN2 used when d_model is not a multiple of 256.
-template <int MODE, int NTW = kChunkRows>
+// GATHER (first GEMM on wide token tiles, e4m3 token rows): the token tile of every stage
+// is copied from the unpermuted activations by four gather warps (16-byte cp.async into
+// the 128-byte swizzled layout) instead of TMA from a permuted copy; stages are then of
+// fixed size.
+template <int MODE, int NTW = kChunkRows, bool GATHER = false>
 struct Cfg {
   // FP4 weights (MXFP4: E2M1, one E8M0 scale per 32 K-elements) with e4m3 tokens: the FP8
   // kernel with the weight operand unpacked by TMA into the e4m3 layout
-  static constexpr bool kW4 = MODE == kFFN1F4 || MODE == kFFN2F4;
-  static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8 || kW4;
+  static constexpr bool kW4 = MODE == kFFN1F4 || MODE == kFFN2F4 || MODE == kFFN2F4M256;
+  static constexpr bool kFP8 = MODE == kFFN1F8 || MODE == kFFN2F8 || MODE == kFFN2F8M256 || kW4;
   static constexpr bool kGLU = MODE == kFFN1 || MODE == kFFN1F8 || MODE == kFFN1F4;  // gate + up
   static constexpr bool kSecond = MODE == kFFN2 || MODE == kFFN2M256 || MODE == kFFN2M512 ||
-                                  MODE == kFFN2F8 || MODE == kFFN2F4;   // reads h (output rows)
+                                  MODE == kFFN2F8 || MODE == kFFN2F4 || MODE == kFFN2F8M256 ||
+                                  MODE == kFFN2F4M256;   // reads h (output rows)
   // FFN2: 128-row weight blocks (= 128 output columns each) per tile
-  static constexpr int kOutBlocks = MODE == kFFN2M512 ? 4 : (MODE == kFFN2M256 ? 2 : 1);
+  static constexpr int kOutBlocks =
+      MODE == kFFN2M512 ? 4
+                        : ((MODE == kFFN2M256 || MODE == kFFN2F8M256 || MODE == kFFN2F4M256) ? 2 : 1);
   static_assert(NTW == kChunkRows || MODE != kRouter, "router tiles are 128 tokens wide");
   static constexpr int kATiles = kGLU ? 2 : kOutBlocks;             // weight tiles per stage
   // FP8 tiles: 112 tokens (112 / 224 are passed in as NTW), leaving TMEM room for the
@@ -122,7 +134,11 @@ struct Cfg {
   static constexpr uint32_t kColsUsed = kAccBufs * kAccCols + kSFCols;
   static constexpr uint32_t kTmemCols =
       kColsUsed <= 64 ? 64 : (kColsUsed <= 128 ? 128 : (kColsUsed <= 256 ? 256 : 512));
-  static constexpr int kThreads = kFP8 ? 224 : 192;                 // + one scale-factor warp
+  static constexpr int kGatherWarp0 = kFP8 ? 7 : 6;                 // first gather warp
+  static constexpr int kGatherThreads = 128;
+  // + one scale-factor warp (FP8), + four gather warps (GATHER)
+  static constexpr int kThreads = (kFP8 ? 224 : 192) + (GATHER ? kGatherThreads : 0);
+  static constexpr bool kFixedStages = kFP8 || GATHER;
   static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;      // per epilogue warp: 16 x 32 x 4 B
   static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;   // group (half-)chunk prefixes
   static constexpr uint32_t kRedBytes = kFP8 ? 2 * 4 * 128 * 4 : 0;  // FP8 amax exchange
@@ -131,9 +147,9 @@ struct Cfg {
   // filling the rest of shared memory.
   static constexpr uint32_t kFixedBytes = 1024 /*barriers*/ + kStagingBytes + kGrpBytes + 16 +
                                           kRedBytes + 1024 /*align*/;
-  static constexpr int kSlots = kFP8 ? kStages : kRingSlots;
+  static constexpr int kSlots = kFixedStages ? kStages : kRingSlots;
   static constexpr uint32_t kRingBytes =
-      kFP8 ? kStages * kStageBytes : ((kMaxSmem - kFixedBytes) / 1024) * 1024;
+      kFixedStages ? kStages * kStageBytes : ((kMaxSmem - kFixedBytes) / 1024) * 1024;
   static constexpr uint32_t kSmemBytes = kRingBytes + kFixedBytes;
   static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
   static_assert(kColsUsed <= 512, "TMEM budget");
@@ -218,17 +234,6 @@ __device__ __forceinline__ Chunk tile_rows(const DevParams& p, const TileCoord& 
   return c;
 }
 
-// Smallest e with amax <= 448 * 2^e (amax as fp32 bits, non-negative), clamped to the
-// UE8M0 range: the power-of-two scale of an e4m3 block.  448 = 1.75 * 2^8, so with
-// amax = m * 2^ea (m in [1, 2)): e = ea - 8 when m <= 1.75, else ea - 7.
-__device__ __forceinline__ int e4m3_scale_exponent(uint32_t amax_bits) {
-  if (amax_bits == 0) return 0;
-  const int ea = static_cast<int>((amax_bits >> 23) & 0xFFu);
-  if (ea == 0) return -127;
-  const int e = (ea - 127) - ((amax_bits & 0x7FFFFFu) <= 0x600000u ? 8 : 7);
-  return max(-127, min(127, e));
-}
-
 // Pipeline stages of variable size in a byte ring of shared memory.  A stage takes the
 // bytes right after the previous stage's, or offset 0 when it would run past the end of
 // the ring, so a tile of few tokens keeps more K blocks of weights in flight than a tile
@@ -297,10 +302,10 @@ __device__ __forceinline__ void store_block_16x32(T* g, int ld, int nvalid, cons
   __syncwarp();
 }
 
-template <int MODE, int NTW>
-__global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
+template <int MODE, int NTW, bool GATHER>
+__global__ void __launch_bounds__(Cfg<MODE, NTW, GATHER>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ DevParams p) {
-  using C = Cfg<MODE, NTW>;
+  using C = Cfg<MODE, NTW, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -324,7 +329,8 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kSlots; ++i) {
-      mbar_init(&full_bar[i], C::kFP8 ? 1 + 32 : 1);
+      // the producer's expect-tx arrive, + the scale warp's lanes, + the gather threads
+      mbar_init(&full_bar[i], 1 + (C::kFP8 ? 32 : 0) + (GATHER ? C::kGatherThreads : 0));
       mbar_init(&empty_bar[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -374,8 +380,9 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
         const int tok_row = C::kSecond ? c.o_row : c.b_row;
         // TMA bytes per stage: a packed FP4 weight box lands unpacked (16 KB of shared memory)
         // but completes its packed size in bytes (8 KB) on the barrier
-        const uint32_t bytes = C::kATiles * (C::kW4 ? kABytes / 2 : kABytes) + n_pad * kRowBytes;
-        const uint32_t stage_bytes = C::kFP8 ? C::kStageBytes : bytes;     // ring bytes per stage
+        const uint32_t bytes = C::kATiles * (C::kW4 ? kABytes / 2 : kABytes) +
+                               (GATHER ? 0u : static_cast<uint32_t>(n_pad) * kRowBytes);
+        const uint32_t stage_bytes = C::kFixedStages ? C::kStageBytes : bytes;  // ring bytes per stage
         const CUtensorMap* wm = &p.wmap[c.seg];
         for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
           uint32_t slot, soff;
@@ -393,8 +400,8 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           for (int j = 1; j < C::kOutBlocks; ++j)
             tma_load_2d(st + j * kABytes, wm, &full_bar[slot], kx, a_row + j * kBM);
           uint8_t* bt = st + C::kATiles * kABytes;
-          // token rows as boxes of 128 / 64 / 32 / 16 rows covering n_pad
-          for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
+          // token rows as boxes of 128 / 64 / 32 / 16 rows covering n_pad (unless gathered)
+          for (int bi = 0, off = 0; bi < kTokBoxes && !GATHER; ++bi) {
             const int rows = 128 >> bi;
             while (n_pad - off >= rows) {
               tma_load_2d(bt + off * kRowBytes, &p.tmap[c.seg][bi], &full_bar[slot], kx, tok_row + off);
@@ -433,14 +440,17 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           tc_fence_after();
           const uint32_t st = smem_u32(tiles) + slot_off[stage];
           const uint32_t bt = st + C::kATiles * kABytes;
+          // rows written by cp.async (scale atoms, gathered tokens) before the async-proxy reads
+          if (C::kFP8 || GATHER) fence_proxy_async_smem();
           if (C::kFP8) {
             // scale factors of this stage: smem (written by the scale warp) -> TMEM
-            fence_proxy_async_smem();
             const uint32_t sf_smem = bt + C::kBBytes;
             const uint32_t sfa = tmem_base + C::kAccBufs * C::kAccCols + stage * C::kSFColsPerStage;
             const uint32_t sfb = sfa + C::kATiles * 4;
-            tmem_cp_32x128b_warpx4(sfa, smem_desc_noswizzle(sf_smem));
-            if (C::kGLU) tmem_cp_32x128b_warpx4(sfa + 4, smem_desc_noswizzle(sf_smem + kSFAtomBytes));
+            // weight-side scales: one atom per weight tile (gate and up, or output blocks)
+#pragma unroll
+            for (int j = 0; j < C::kATiles; ++j)
+              tmem_cp_32x128b_warpx4(sfa + 4 * j, smem_desc_noswizzle(sf_smem + j * kSFAtomBytes));
             // token-side scales: one atom per 128 token rows, in consecutive 4-column groups
 #pragma unroll
             for (int a = 0; a < C::kSFBAtoms; ++a)
@@ -451,10 +461,10 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
               const uint32_t accum = (kb > tc.kb0 || kk) ? 1u : 0u;
               const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
               const uint32_t id = C::kW4 ? (idesc_w4 | (static_cast<uint32_t>(kk) << 29)) : idesc;
-              umma_e4m3_bs(d0, umma_desc_sw128(st + kk * 32), bdesc, id, sfa, sfb, accum);
-              if (C::kGLU)
-                umma_e4m3_bs(d1, umma_desc_sw128(st + kABytes + kk * 32), bdesc, id, sfa + 4, sfb,
-                             accum);
+#pragma unroll
+              for (int j = 0; j < C::kATiles; ++j)
+                umma_e4m3_bs(d0 + j * C::kNT, umma_desc_sw128(st + j * kABytes + kk * 32), bdesc, id,
+                             sfa + 4 * j, sfb, accum);
             }
           } else {
 #pragma unroll
@@ -554,7 +564,8 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
                                 static_cast<size_t>(c.o_row + n0) * p.ld_out + (m - lane),
                             p.ld_out, c.nrows - n0, hv,
                             reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
-        } else if (MODE == kFFN2M256 || MODE == kFFN2M512) {
+        } else if (MODE == kFFN2M256 || MODE == kFFN2M512 || MODE == kFFN2F8M256 ||
+                   MODE == kFFN2F4M256) {
           // accumulator j holds output columns (mb * kOutBlocks + j) * 128 + (0..127)
           __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
                                 (mb * C::kOutBlocks * kBM + m_local - lane);
@@ -597,14 +608,13 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
       mbar_arrive(&tempty_bar[acc]);
       ++it;
     }
-  } else if (C::kFP8) {
+  } else if (C::kFP8 && warp == 6) {
     // ------------------------------------------------------------ scale-factor warp (FP8)
     // Per stage: the 512-byte scale atoms of the weight tile(s) and of the token rows (row
     // n's 4 bytes at (n % 32) * 16 + (n / 32) * 4), copied with cp.async; each lane's
     // completion arrives on the stage's full barrier.  e4m3 weights: one UE8M0 value for
     // the whole 128x128 block, replicated.  FP4 weights: row r's 4 bytes are its E8M0
-    // scales of the stage's four 32-element K runs, read straight from the caller's
-    // [rows][K / 32] codes.
+    // scales of the stage's four 32-element K runs, copied from the caller's atoms.
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     const int up_rb = p.up_offset / kBM;
@@ -619,6 +629,18 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
                                 : p.wsf[c.seg] + static_cast<size_t>(c.group) * p.wsf_rb_per_group * p.k_blocks;
       const uint32_t* tsf = p.tsf[c.seg];
       const int tld = p.tsf_ld[c.seg], trows = p.tsf_rows[c.seg];
+      // the scale row of each of this lane's token rows, looked up once per tile
+      int trow[4 * C::kSFBAtoms];
+#pragma unroll
+      for (int j = 0; j < 4 * C::kSFBAtoms; ++j) {
+        const int n = lane + 32 * j;
+        trow[j] = min(tok_row + n, trows - 1);
+        if (GATHER) {                      // the token's own row of the unpermuted scales
+          const int32_t* gi = p.gidx[c.seg];
+          const int src = c.b_row + min(n, c.nrows - 1);
+          trow[j] = gi ? __ldg(gi + src) : src;
+        }
+      }
       for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
         const bool w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w)) {
@@ -626,31 +648,92 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW>::kThreads, 1)
           break;
         }
         uint8_t* sf = tiles + stage * C::kStageBytes + C::kATiles * kABytes + C::kBBytes;
-        if (C::kW4) {
-          const uint8_t* wsc = p.wsc[c.seg] +
-              (static_cast<size_t>(c.group) * p.w_rows_per_group + mb * kBM) * p.wsc_ld + kb * 4;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            cp_async_4(sf + lane * 16 + j * 4, wsc + static_cast<size_t>(j * 32 + lane) * p.wsc_ld);
-            if (C::kGLU)
-              cp_async_4(sf + kSFAtomBytes + lane * 16 + j * 4,
-                         wsc + static_cast<size_t>(p.up_offset + j * 32 + lane) * p.wsc_ld);
+        for (int j = 0; j < C::kATiles; ++j) {
+          // 128-row block of the weight matrix behind weight tile j: gate / up rows, or
+          // consecutive output blocks
+          const int rb = C::kGLU ? (j ? up_rb + mb : mb) : mb * C::kOutBlocks + j;
+          if (C::kW4) {
+            // the caller's atoms are already in the layout tcgen05.cp reads: 16 bytes per lane
+            const uint4* wsc = p.wsc[c.seg] + static_cast<size_t>(c.group) * p.wsf_rb_per_group * p.k_blocks * 32;
+            cp_async_16(sf + j * kSFAtomBytes + lane * 16,
+                        wsc + (static_cast<size_t>(rb) * p.k_blocks + kb) * 32 + lane);
+          } else {
+            cp_async_16(sf + j * kSFAtomBytes + lane * 16, wsf + static_cast<size_t>(rb) * p.k_blocks + kb);
           }
-        } else {
-          cp_async_16(sf + lane * 16, wsf + static_cast<size_t>(mb) * p.k_blocks + kb);
-          if (C::kGLU)
-            cp_async_16(sf + kSFAtomBytes + lane * 16,
-                        wsf + static_cast<size_t>(up_rb + mb) * p.k_blocks + kb);
         }
         uint8_t* sfb = sf + C::kATiles * kSFAtomBytes;
 #pragma unroll
         for (int j = 0; j < 4 * C::kSFBAtoms; ++j) {
           const int n = lane + 32 * j;     // atom j / 4, in-atom row group j % 4
           if (n < n_pad) {
-            const int row = min(tok_row + n, trows - 1);
+            const int row = trow[j];
             cp_async_4(sfb + (j >> 2) * kSFAtomBytes + lane * 16 + (j & 3) * 4,
                        tsf + static_cast<size_t>(kb) * tld + row);
           }
+        }
+        cp_async_mbar_arrive_noinc(&full_bar[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (GATHER && warp >= C::kGatherWarp0) {
+    // ------------------------------------------------------------ gather warps
+    // Per stage: the tile's token rows, 128 bytes of K each, copied from the unpermuted
+    // activations with 16-byte cp.async into the 128-byte swizzled layout (16-byte chunk j
+    // of row n at n * 128 + ((j ^ (n % 8)) * 16), as TMA's 128-byte swizzle places it).
+    // Thread g copies chunk g % 8 of rows g / 8 + 16 i: a warp instruction covers four
+    // whole 128-byte rows.  Padding rows (past the chunk's rows) are not copied: their
+    // products land only in output rows that are never stored.  Each thread's completion
+    // arrives on the stage's full barrier.
+    const int g = threadIdx.x - C::kGatherWarp0 * 32;
+    const int j = g & 7, r0 = g >> 3;
+    constexpr int kRowsPerThread = (C::kNT + 15) / 16;
+    // source rows of this thread's token rows in the tile: looked up one tile ahead, so
+    // that the index loads' latency hides behind the previous tile's stages
+    auto rows_of = [&](int t, int (&rows)[kRowsPerThread], Chunk& c, TileCoord& tc) {
+      tc = tile_coord(p, t, grp_cp, n_grp);
+      c = tile_rows<MODE, NTW>(p, tc);
+      const int32_t* gi = c.nrows > 0 ? p.gidx[c.seg] : nullptr;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int n = r0 + 16 * i;
+        rows[i] = n < c.nrows ? (gi ? __ldg(gi + c.b_row + n) : c.b_row + n) : 0;
+      }
+    };
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    int rows[kRowsPerThread], next_rows[kRowsPerThread];
+    Chunk c, next_c;
+    TileCoord tc, next_tc;
+    if (blockIdx.x < n_tiles) rows_of(blockIdx.x, next_rows, next_c, next_tc);
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      c = next_c;
+      tc = next_tc;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) rows[i] = next_rows[i];
+      if (t + static_cast<int>(gridDim.x) < n_tiles)
+        rows_of(t + gridDim.x, next_rows, next_c, next_tc);
+      if (c.nrows <= 0) continue;
+      const uint8_t* src[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i)
+        src[i] = p.gsrc[c.seg] + static_cast<size_t>(rows[i]) * p.g_ld + j * 16;
+      for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
+        const bool w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        uint8_t* bt = tiles + stage * C::kStageBytes + C::kATiles * kABytes;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int n = r0 + 16 * i;
+          if (n < c.nrows)
+            cp_async_16_cg(bt + n * kRowBytes + ((j ^ (n & 7)) << 4), src[i] + kb * kRowBytes);
         }
         cp_async_mbar_arrive_noinc(&full_bar[stage]);
         if (++stage == C::kStages) {
@@ -792,9 +875,9 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
   return cudaGetLastError();
 }
 
-template <int MODE, int NTW>
+template <int MODE, int NTW, bool GATHER = false>
 static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
-  using C = Cfg<MODE, NTW>;
+  using C = Cfg<MODE, NTW, GATHER>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
   DevParams p;
   for (int i = 0; i < 2; ++i) p.wmap[i] = g.wmap[i];
@@ -825,10 +908,14 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
     p.tsf_rows[i] = g.tsf_rows[i];
   }
   p.wsf_rb_per_group = g.wsf_rb_per_group;
-  p.wsc_ld = g.wsc_ld;
   p.out_sf = g.out_sf;
   p.ld_out_sf = g.ld_out_sf;
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, NTW>,
+  for (int i = 0; i < 2; ++i) {
+    p.gsrc[i] = static_cast<const uint8_t*>(g.gsrc[i]);
+    p.gidx[i] = g.gidx[i];
+  }
+  p.g_ld = g.g_ld;
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, NTW, GATHER>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::kSmemBytes));
   if (err != cudaSuccess) return err;
@@ -838,7 +925,7 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
     if (tiles < grid) grid = tiles;
     if (grid == 0) return cudaSuccess;
   }
-  grouped_gemm_kernel<MODE, NTW><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
+  grouped_gemm_kernel<MODE, NTW, GATHER><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -859,13 +946,17 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
     // kChunkRowsFP8); the second GEMM takes 224-token tiles once chunks are 224 rows
     case kFFN1F8:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1F8, kChunkRowsNarrow>(g, s);
+      if (g.gather) return launch_mode<kFFN1F8, kChunkRows, true>(g, s);
       return launch_mode<kFFN1F8, kChunkRows>(g, s);
     case kFFN2F8:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2F8, kChunkRowsNarrow>(g, s);
       if (g.tile_tokens == 2 * kChunkRowsFP8) return launch_mode<kFFN2F8, 2 * kChunkRowsFP8>(g, s);
       return launch_mode<kFFN2F8, kChunkRows>(g, s);
+    case kFFN2F8M256: return launch_mode<kFFN2F8M256, kChunkRowsNarrow>(g, s);
+    case kFFN2F4M256: return launch_mode<kFFN2F4M256, kChunkRowsNarrow>(g, s);
     case kFFN1F4:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1F4, kChunkRowsNarrow>(g, s);
+      if (g.gather) return launch_mode<kFFN1F4, kChunkRows, true>(g, s);
       return launch_mode<kFFN1F4, kChunkRows>(g, s);
     case kFFN2F4:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN2F4, kChunkRowsNarrow>(g, s);

@@ -68,6 +68,23 @@ cudaError_t launch_permute(const int32_t* topk_idx, int T, int E, int k, const v
                            cudaStream_t s);
 inline int permute_chunks(int T) { return (T + 255) / 256; }
 
+// The routing tables of the permutation alone (group offsets, perm_token, inv_perm): the
+// count (+ rank) kernels, no row copy.
+cudaError_t launch_permute_index(const int32_t* topk_idx, int T, int E, int k, int32_t* perm_token,
+                                 int32_t* inv_perm, int32_t* offsets, int32_t* chunk_counts,
+                                 unsigned* done, int* status, cudaStream_t s);
+
+// The permutation of bf16 rows [T, d] into e4m3 rows for e4m3 expert GEMMs, quantised in
+// the copy (one power-of-two scale per token per 128 values, round to nearest even).  Block
+// scales go to x_perm_scale ([T k][d/128] fp32) when it is non-null, else to x_perm_w as
+// UE8M0 words ([d/128][T k]); x_q / x_q_w (both or neither): every token's own quantised
+// row [T, d] and scale words [d/128][T].  x_perm null: only x_q / x_q_w are written.
+cudaError_t launch_permute_quant(const int32_t* topk_idx, int T, int E, int k, const void* x_bf16,
+                                 int d, void* x_perm, float* x_perm_scale, uint32_t* x_perm_w,
+                                 void* x_q, uint32_t* x_q_w, int32_t* perm_token, int32_t* inv_perm,
+                                 int32_t* offsets, int32_t* chunk_counts, unsigned* done,
+                                 int* status, cudaStream_t s);
+
 // Tile planner: routed groups (device offsets [G+1], rows <= n_rows) followed
 // by n_shared groups of T rows each (token rows 0..T-1 of the unpermuted
 // activations, output rows shared_o_row + s*T).  Heavy groups first.
@@ -80,9 +97,10 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
 
 // kFFN2M256 / kFFN2M512: FFN2 (bf16) with 256 / 512 weight rows per tile, as two / four
 // 128-row blocks (M512: decode-sized token tiles only).  kFFN1F4 / kFFN2F4: the FP8 GEMMs
-// with FP4 (MXFP4) weights.
+// with FP4 (MXFP4) weights.  kFFN2F8M256 / kFFN2F4M256: FP8 / FP4 FFN2 with two 128-row
+// weight blocks per tile (decode-sized token tiles).
 enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5,
-                kFFN2M512 = 6, kFFN1F4 = 7, kFFN2F4 = 8 };
+                kFFN2M512 = 6, kFFN1F4 = 7, kFFN2F4 = 8, kFFN2F8M256 = 9, kFFN2F4M256 = 10 };
 
 struct GemmLaunch {
   int mode;
@@ -113,9 +131,15 @@ struct GemmLaunch {
   // the scales of its requantised output to out_sf ([I / 128][ld_out_sf]).
   const uint4* wsf[2];
   int wsf_rb_per_group;
-  // FP4 modes: E8M0 weight scale codes per segment, [rows][K / 32] (wsc_ld = K / 32)
-  const uint8_t* wsc[2];
-  int wsc_ld;
+  // gather-on-load (first GEMM, wide token tiles): token row n of a chunk is row
+  // gidx[seg][b_row + n] (gidx null: b_row + n) of gsrc[seg], g_ld bytes apart
+  bool gather;
+  const void* gsrc[2];
+  const int32_t* gidx[2];
+  int g_ld;
+  // FP4 modes: E8M0 weight scale codes per segment in 512-byte atoms
+  // [groups][rows / 128][K / 128][32 x 16 bytes] (row r, K run q at (r % 32) * 16 + (r / 32) * 4 + q)
+  const uint4* wsc[2];
   const uint32_t* tsf[2];
   int tsf_ld[2];
   int tsf_rows[2];

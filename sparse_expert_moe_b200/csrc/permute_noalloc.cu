@@ -57,6 +57,9 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
     return MOE_ERR_INVALID_ARG;
+  // bf16 rows for e4m3 / FP4 experts are quantised by moe_permute; not on this path
+  if (cfg->act == MOE_BF16 && (cfg->weight == MOE_E4M3 || cfg->weight == MOE_E2M1))
+    return MOE_ERR_UNSUPPORTED;
   // e4m3 rows come with one fp32 scale per 128 channels, permuted alongside the rows
   const bool fp8 = cfg->act == MOE_E4M3;
   if (fp8 && cfg->T > 0 && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;

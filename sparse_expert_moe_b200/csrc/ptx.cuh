@@ -23,6 +23,17 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Smallest e with amax <= 448 * 2^e (amax as fp32 bits, non-negative), clamped to the
+// UE8M0 range: the power-of-two scale of an e4m3 block.  448 = 1.75 * 2^8, so with
+// amax = m * 2^ea (m in [1, 2)): e = ea - 8 when m <= 1.75, else ea - 7.
+__device__ __forceinline__ int e4m3_scale_exponent(uint32_t amax_bits) {
+  if (amax_bits == 0) return 0;
+  const int ea = static_cast<int>((amax_bits >> 23) & 0xFFu);
+  if (ea == 0) return -127;
+  const int e = (ea - 127) - ((amax_bits & 0x7FFFFFu) <= 0x600000u ? 8 : 7);
+  return max(-127, min(127, e));
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -220,6 +231,12 @@ __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src)
 }
 __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+// 16-byte copy cached in L2 only (not L1): for data each SM reads once per stage.
+__device__ __forceinline__ void cp_async_16_cg(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
                "l"(gmem_src)
                : "memory");
 }

@@ -30,6 +30,8 @@ More, Smaller Experts" -- 384 experts, top-8 plus one shared expert):
   r1_decode_fp8   r1_decode with e4m3 activations and e4m3 weights
   r1_decode_fp4   r1_decode with e4m3 activations and MXFP4 weights (E2M1 codes, one E8M0
                   scale per 32 elements along K)
+  r1_decode_fp4q  r1_decode (bf16 activations) with MXFP4 weights: the activations are
+                  quantised to e4m3 in the permutation
 """
 from __future__ import annotations
 
@@ -89,6 +91,8 @@ SPECS = {
                           "e4m3", "bf16", family="r1", x_stream=2, bias_range=0.1),
     "r1_decode_fp4": Spec("r1_decode_fp4", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
                           "e2m1", "bf16", family="r1", x_stream=2, bias_range=0.1),
+    "r1_decode_fp4q": Spec("r1_decode_fp4q", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "bf16",
+                           "e2m1", "bf16", family="r1", x_stream=2, bias_range=0.1),
     "r1_prefill_fp8": Spec("r1_prefill_fp8", 8192, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
                            "e4m3", "bf16", family="r1", x_stream=3, loads="zipf"),
 }
@@ -160,6 +164,23 @@ def to_mxfp4(a: np.ndarray, block: int = 32):
     return torch.from_numpy(packed), torch.from_numpy((e + 127).astype(np.uint8))
 
 
+def scale_atoms(codes):
+    """E8M0 codes [R, K/32] -> the ABI's scale atoms [R/128, K/128, 512]: row r, run q of an
+    atom at byte (r % 32) * 16 + (r / 32) * 4 + q (a pure reordering of the bytes)."""
+    c = np.asarray(codes, np.uint8)
+    R, Q = c.shape
+    a = c.reshape(R // 128, 4, 32, Q // 4, 4)           # [rb, r / 32, r % 32, kb, q]
+    return torch.from_numpy(np.ascontiguousarray(a.transpose(0, 3, 2, 1, 4)).reshape(R // 128, Q // 4, 512))
+
+
+def scale_rows(atoms):
+    """The inverse of scale_atoms: [R/128, K/128, 512] -> [R, K/32]."""
+    a = np.asarray(atoms, np.uint8)
+    RB, KB, _ = a.shape
+    b = a.reshape(RB, KB, 32, 4, 4).transpose(0, 3, 2, 1, 4)   # [rb, r / 32, r % 32, kb, q]
+    return torch.from_numpy(np.ascontiguousarray(b).reshape(RB * 128, KB * 4))
+
+
 # ---------------------------------------------------------------------------
 # draws
 # ---------------------------------------------------------------------------
@@ -196,7 +217,8 @@ def _encode_weight(spec: Spec, w32: np.ndarray):
     if spec.weight == "e4m3":
         return to_e4m3_blocks(w32, 128, 128)
     if spec.weight == "e2m1":
-        return to_mxfp4(w32)
+        q, s = to_mxfp4(w32)
+        return q, scale_atoms(s.numpy())
     raise ValueError(spec.weight)
 
 
@@ -252,9 +274,14 @@ def draw_logits(T: int, E: int, seed: int, lo=-3.0, hi=3.0, redraw=None, stream=
     """fp32 router logits U(lo, hi) supplied directly to the routing kernels."""
     L = _rng(seed, _FAMILY["custom"], _LOGITS, stream, T, E).uniform(lo, hi, (T, E)).astype(np.float32)
     for t, attempt in (redraw or []):
-        L[t] = _rng(seed, _FAMILY["custom"], _LOGITS, stream, T, E, t, attempt).uniform(
-            lo, hi, E).astype(np.float32)
+        L[t] = draw_logit_row(T, E, seed, t, attempt, lo, hi, stream)
     return L
+
+
+def draw_logit_row(T: int, E: int, seed: int, t: int, attempt: int, lo=-3.0, hi=3.0, stream=0):
+    """Replacement draw number ``attempt`` (>= 1) for row t of ``draw_logits``."""
+    return _rng(seed, _FAMILY["custom"], _LOGITS, stream, T, E, t, attempt).uniform(
+        lo, hi, E).astype(np.float32)
 
 
 # ---------------------------------------------------------------------------
@@ -282,11 +309,11 @@ class Workload:
 
 def _stack_experts(spec, seed, n, shared, threads):
     I, d = spec.d_ff, spec.d_model
-    if spec.weight == "e2m1":          # packed codes [rows, K/2] + E8M0 codes [rows, K/32]
+    if spec.weight == "e2m1":          # packed codes [rows, K/2] + E8M0 scale atoms
         w13 = torch.empty((n, 2 * I, d // 2), dtype=torch.uint8)
         w2 = torch.empty((n, d, I // 2), dtype=torch.uint8)
-        s13 = torch.empty((n, 2 * I, d // 32), dtype=torch.uint8)
-        s2 = torch.empty((n, d, I // 32), dtype=torch.uint8)
+        s13 = torch.empty((n, 2 * I // 128, d // 128, 512), dtype=torch.uint8)
+        s2 = torch.empty((n, d // 128, I // 128, 512), dtype=torch.uint8)
         scaled = True
     else:
         wdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[spec.weight]

@@ -73,6 +73,10 @@ def load_library() -> ctypes.CDLL:
         "moe_read_device_status": [P, P, ctypes.POINTER(ctypes.c_int)],
         "moe_reset_device_status": [P, P],
         "moe_selftest_bounded_wait": [P, ctypes.c_longlong, P],
+        "moe_layer_graph_create": [cfgp, ctypes.POINTER(MoeWeights), P, P, P, P, P, P, SZ,
+                                   ctypes.POINTER(ctypes.c_void_p)],
+        "moe_layer_graph_launch": [P, P],
+        "moe_layer_graph_destroy": [P],
     }
     for name, argtypes in sigs.items():
         fn = getattr(lib, name)
@@ -195,6 +199,33 @@ def moe_layer_forward_staged(cfg, weights: MoeWeights, x, x_scale, y, topk_idx_o
     _check("moe_layer_forward_staged", load_library().moe_layer_forward_staged(
         ctypes.byref(cfg), ctypes.byref(weights), _p(x), _p(x_scale), _p(y), _p(topk_idx_out),
         _p(topk_w_out), _p(ws), ws.numel() * ws.element_size(), _stream(stream), handles))
+
+
+class LayerGraph:
+    """moe_layer_graph_create / _launch / _destroy: the layer recorded once for fixed
+    tensors (x, y, routing outputs, workspace) and replayed with one graph launch."""
+
+    def __init__(self, cfg, weights: MoeWeights, x, x_scale, y, topk_idx_out, topk_w_out, ws):
+        h = ctypes.c_void_p(0)
+        _check("moe_layer_graph_create", load_library().moe_layer_graph_create(
+            ctypes.byref(cfg), ctypes.byref(weights), _p(x), _p(x_scale), _p(y), _p(topk_idx_out),
+            _p(topk_w_out), _p(ws), ws.numel() * ws.element_size(), ctypes.byref(h)))
+        self._h = h
+        self._keep = (cfg, weights, x, x_scale, y, topk_idx_out, topk_w_out, ws)
+
+    def launch(self, stream=None):
+        _check("moe_layer_graph_launch", load_library().moe_layer_graph_launch(self._h, _stream(stream)))
+
+    def close(self):
+        if self._h:
+            _check("moe_layer_graph_destroy", load_library().moe_layer_graph_destroy(self._h))
+            self._h = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def moe_read_device_status(ws, stream=None) -> int:

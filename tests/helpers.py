@@ -27,17 +27,20 @@ def topk_gaps(keys, k):
 
 
 def margin_logits(T, E, k, score, bias, margin=1e-3, seed=0, stream=0):
-    """U(-3, 3) fp32 logits whose rows are redrawn until the top k+1 keys are >= margin apart."""
-    redraw = {}
-    while True:
-        L = inputs.draw_logits(T, E, seed, redraw=sorted(redraw.items()), stream=stream)
-        keys = oracle.selection_keys(L.astype(np.float64), score,
-                                     None if bias is None else np.asarray(bias, np.float64))
-        bad = np.nonzero(topk_gaps(keys, k) < margin)[0]
-        if bad.size == 0:
-            return L
+    """U(-3, 3) fp32 logits whose rows are redrawn until the top k+1 keys are >= margin apart
+    (``inputs.draw_logits`` with those redraws; only the failing rows are redrawn and
+    re-checked each round)."""
+    b64 = None if bias is None else np.asarray(bias, np.float64)
+    L = inputs.draw_logits(T, E, seed, stream=stream)
+    attempts = np.zeros(T, np.int64)
+    bad = np.arange(T)
+    while bad.size:
+        keys = oracle.selection_keys(L[bad].astype(np.float64), score, b64)
+        bad = bad[topk_gaps(keys, k) < margin]
         for t in bad:
-            redraw[int(t)] = redraw.get(int(t), 0) + 1
+            attempts[t] += 1
+            L[t] = inputs.draw_logit_row(T, E, seed, int(t), int(attempts[t]), stream=stream)
+    return L
 
 
 def act_values(wl) -> np.ndarray:
@@ -104,8 +107,8 @@ def dequant_mxfp4_fast(packed, scale_codes):
 def _w_values(w, s, shape_blocks):
     if s is None:
         return w.double().numpy()
-    if s.dtype == torch.uint8:          # MXFP4: packed E2M1 + E8M0 codes
-        return dequant_mxfp4_fast(w.numpy(), s.numpy())
+    if s.dtype == torch.uint8:          # MXFP4: packed E2M1 + E8M0 scale atoms
+        return dequant_mxfp4_fast(w.numpy(), inputs.scale_rows(s.numpy()).numpy())
     return dequant_fast(w.view(torch.uint8).numpy(), s.numpy(), 128, 128)
 
 
@@ -153,5 +156,16 @@ def oracle_layer(wl, rows=None, return_routing=False):
             _w_values(wl.ws13[s], None if wl.ws13_s is None else wl.ws13_s[s], None),
             _w_values(wl.ws2[s], None if wl.ws2_s is None else wl.ws2_s[s], None))))
     bias = None if wl.sel_bias is None else wl.sel_bias.double().numpy()
+    expert_x = None
+    if spec.act == "bf16" and spec.weight in ("e4m3", "e2m1"):
+        # bf16 activations into e4m3 / FP4 experts: the experts take x quantised to e4m3
+        expert_x = quantised_values(xv)
     return oracle.layer_forward(xv, wl.wr.double().numpy(), spec.score, spec.top_k, expert, spec.E,
-                                shared, sel_bias=bias, return_routing=return_routing)
+                                shared, sel_bias=bias, return_routing=return_routing,
+                                expert_x=expert_x)
+
+
+def quantised_values(x):
+    """The values of the oracle's e4m3 block quantisation of x (1 x 128 blocks)."""
+    codes, sc = oracle.quantize_e4m3_blocks(x)
+    return dequant_fast(codes, sc, 1, 128)

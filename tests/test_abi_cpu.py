@@ -73,6 +73,33 @@ def test_null_pointers_rejected_before_launch(lib):
                                None, None, 0, None) == 1
 
 
+def test_layer_graph_argument_checks(lib):
+    """moe_layer_graph_create checks its arguments before recording anything; destroying a
+    null handle is a no-op and launching one is rejected."""
+    cfg = moe.make_config(16, 256, 8, 2, 256, 0)
+    fake = 256
+    w = moe.MoeWeights(fake, 0, fake, fake, 0, 0, 0, 0, 0, 0)
+    h = ctypes.c_void_p(0)
+    assert lib.moe_layer_graph_create(ctypes.byref(cfg), ctypes.byref(w), fake, None, fake, None,
+                                      None, fake, 1024, None) == 1          # no handle pointer
+    assert lib.moe_layer_graph_create(ctypes.byref(cfg), ctypes.byref(w), fake, None, fake, None,
+                                      None, fake, 1024, ctypes.byref(h)) == 3  # workspace
+    assert lib.moe_layer_graph_create(ctypes.byref(cfg), None, fake, None, fake, None, None, fake,
+                                      1 << 30, ctypes.byref(h)) == 1
+    assert h.value is None
+    assert lib.moe_layer_graph_destroy(None) == 0
+    assert lib.moe_layer_graph_launch(None, None) == 1
+
+
+def test_noalloc_rejects_the_quantising_permutation(lib):
+    """bf16 rows for e4m3 / FP4 experts are quantised by moe_permute only."""
+    fake = 256
+    for weight in ("e4m3", "e2m1"):
+        cfg = moe.make_config(16, 256, 8, 2, 256, 0, act="bf16", weight=weight)
+        assert lib.moe_permute_noalloc(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, fake,
+                                       fake, None) == 2
+
+
 def test_workspace_too_small_rejected(lib):
     cfg = moe.make_config(16, 256, 8, 2, 256, 0)
     fake = 256  # a non-null, 16-byte-aligned address; never dereferenced on this path

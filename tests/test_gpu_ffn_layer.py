@@ -219,6 +219,37 @@ def test_layer_custom(T, d, E, k, I, S, score):
     _check_layer(margin_workload(spec, seed=T))
 
 
+@pytest.mark.parametrize("act", ["bf16", "e4m3"])
+def test_layer_graph_replays_match_eager(act):
+    """The layer recorded as a CUDA graph gives moe_layer_forward's results bit for bit, and
+    a replay after new activations are written into x computes on the new values."""
+    spec = inputs.custom_spec(96, 512, 16, 4, 256, 1, act=act, weight=act)
+    wl = margin_workload(spec, seed=12)
+    layer = moe.DeviceLayer.from_workload(wl, DEV)
+    x = (wl.x.view(torch.uint8) if act == "e4m3" else wl.x).to(DEV)
+    xv = x.view(torch.float8_e4m3fn) if act == "e4m3" else x
+    xs = None if wl.x_scale is None else wl.x_scale.to(DEV)
+    T, k = spec.T, spec.top_k
+    y_g, y_e = layer.output(DEV), layer.output(DEV)
+    idx_g = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gw_g = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    graph = moe.LayerGraph(layer.cfg, layer.weights, xv, xs, y_g, idx_g, gw_g, layer.ws)
+    other = x.flip(0).clone()
+    for step in range(2):
+        if step == 1:
+            x.copy_(other)                 # new activations, same buffer
+        graph.launch()
+        torch.cuda.synchronize()
+        g = (y_g.clone(), idx_g.clone(), gw_g.clone())
+        idx_e = torch.empty_like(idx_g)
+        gw_e = torch.empty_like(gw_g)
+        layer.forward(xv, xs, y_e, idx_e, gw_e)
+        torch.cuda.synchronize()
+        assert torch.equal(g[0], y_e) and torch.equal(g[1], idx_e) and torch.equal(g[2], gw_e)
+    assert moe.moe_read_device_status(layer.ws) == 0
+    graph.close()
+
+
 def test_layer_is_deterministic():
     spec = inputs.custom_spec(300, 256, 16, 4, 256, 1)
     wl = margin_workload(spec, seed=4)

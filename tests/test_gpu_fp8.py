@@ -123,13 +123,13 @@ def test_grouped_ffn_fp4_weights_vs_oracle(sizes, d, I):
     a, a_s = _e4m3(rng.standard_normal((n_rows, d)) * np.exp2(rng.integers(-3, 3, (n_rows, 1))), 1, 128)
     w13 = [_mxfp4(2 * I, d, rng) for _ in range(G)]
     w2 = [_mxfp4(d, I, rng) for _ in range(G)]
+    atoms = lambda ws: torch.stack([inputs.scale_atoms(s.numpy()) for _, s in ws]).to(DEV)
     cfg = moe.make_config(n_rows, d, G, 1, I, 0, act="e4m3", weight="e2m1")
     ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
     y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
     moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows, a.view(torch.uint8).to(DEV),
-                        a_s.to(DEV), torch.stack([q for q, _ in w13]).to(DEV),
-                        torch.stack([s for _, s in w13]).to(DEV), torch.stack([q for q, _ in w2]).to(DEV),
-                        torch.stack([s for _, s in w2]).to(DEV), y, ws)
+                        a_s.to(DEV), torch.stack([q for q, _ in w13]).to(DEV), atoms(w13),
+                        torch.stack([q for q, _ in w2]).to(DEV), atoms(w2), y, ws)
     assert moe.moe_read_device_status(ws) == 0
     av = _dq(a, a_s, 1, 128)
     ref = np.zeros((n_rows, d))
@@ -141,6 +141,37 @@ def test_grouped_ffn_fp4_weights_vs_oracle(sizes, d, I):
     got = y.float().cpu().numpy()
     assert np.isfinite(got).all()
     assert max_rel_err(got, ref) < TOL_FP8
+
+
+@pytest.mark.parametrize("T,E,k,d", [(300, 32, 4, 256), (64, 8, 2, 128), (1000, 256, 8, 7168)])
+@pytest.mark.parametrize("weight", ["e4m3", "e2m1"])
+def test_permute_quantises_bf16_rows_for_low_precision_experts(T, E, k, d, weight):
+    """bf16 activations with e4m3 / FP4 expert weights: moe_permute quantises the rows to e4m3
+    in the copy -- codes and power-of-two scales equal to the oracle's quantisation, bit for
+    bit, placed by the oracle's permutation."""
+    rng = np.random.default_rng(T + d)
+    idx, _ = oracle.route(rng.uniform(-3, 3, (T, E)), "softmax", k)
+    x32 = rng.standard_normal((T, d)) * np.exp2(rng.integers(-12, 12, (T, d // 128))).repeat(128, 1)
+    x32[0, :128] = 0.0                                   # an all-zero block
+    x = inputs.to_bf16(x32.astype(np.float32))
+    cfg = moe.make_config(T, d, E, k, 128, 0, act="bf16", weight=weight)
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    R = T * k
+    x_perm = torch.zeros((R, d), dtype=torch.uint8, device=DEV)
+    x_perm_s = torch.zeros((R, d // 128), dtype=torch.float32, device=DEV)
+    perm_token = torch.empty(R, dtype=torch.int32, device=DEV)
+    inv_perm = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    moe.moe_permute(cfg, torch.from_numpy(idx.astype(np.int32)).to(DEV), x.to(DEV), None, x_perm,
+                    x_perm_s, perm_token, inv_perm, offsets, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    ro, rp, ri = oracle.permute(idx, E)
+    codes, sc = oracle.quantize_e4m3_blocks(x.double().numpy())
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(perm_token.cpu().numpy(), rp)
+    assert np.array_equal(inv_perm.cpu().numpy(), ri)
+    assert np.array_equal(x_perm.cpu().numpy(), codes[rp])
+    assert np.array_equal(x_perm_s.cpu().numpy().astype(np.float64), sc[rp])
 
 
 def test_permute_fp8_rows_and_scales():
@@ -171,7 +202,8 @@ def _check_fp8_layer(wl, rows=None, routing=None):
     layer = moe.DeviceLayer.from_workload(wl, DEV)
     idx = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.int32, device=DEV)
     gw = torch.empty((layer.cfg.T, layer.cfg.top_k), dtype=torch.float32, device=DEV)
-    y = layer.forward(wl.x.to(DEV), wl.x_scale.to(DEV), topk_idx=idx, topk_w=gw)
+    xs = None if wl.x_scale is None else wl.x_scale.to(DEV)
+    y = layer.forward(wl.x.to(DEV), xs, topk_idx=idx, topk_w=gw)
     torch.cuda.synchronize()
     assert moe.moe_read_device_status(layer.ws) == 0
     got, idx, gw = y.float().cpu().numpy(), idx.cpu().numpy(), gw.cpu().numpy()
@@ -196,8 +228,28 @@ def test_layer_fp8_custom(T, d, E, k, I, S, weight):
     _check_fp8_layer(margin_workload(spec, seed=T + 1))
 
 
+@pytest.mark.parametrize("T,d,E,k,I,S", [(70, 256, 16, 4, 256, 1), (300, 384, 8, 2, 128, 2),
+                                         (1, 128, 4, 1, 128, 1)])
+@pytest.mark.parametrize("weight", ["e4m3", "e2m1"])
+def test_layer_bf16_activations_low_precision_experts(T, d, E, k, I, S, weight):
+    """bf16 activations, e4m3 / FP4 experts: the router takes x as given, the experts take x
+    quantised to e4m3 in the permutation (the oracle applies its own quantisation)."""
+    spec = inputs.custom_spec(T, d, E, k, I, S, act="bf16", weight=weight)
+    wl = margin_workload(spec, seed=T + 3)
+    layer = moe.DeviceLayer.from_workload(wl, DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gw = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    y = layer.forward(wl.x.to(DEV), None, topk_idx=idx, topk_w=gw)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(layer.ws) == 0
+    ref, r = oracle_layer(wl, return_routing=True)
+    assert np.array_equal(idx.cpu().numpy(), r["idx"])
+    np.testing.assert_allclose(gw.cpu().numpy(), r["gates"], rtol=1e-5, atol=1e-6)
+    assert max_rel_err(y.float().cpu().numpy(), ref) < TOL_FP8
+
+
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["r1_decode_fp8", "r1_decode_fp4"])
+@pytest.mark.parametrize("name", ["r1_decode_fp8", "r1_decode_fp4", "r1_decode_fp4q"])
 def test_layer_r1_decode_low_precision_full(name):
     """The DeepSeek-R1 decode layer with e4m3 activations and e4m3 or MXFP4 weights, every
     token checked."""

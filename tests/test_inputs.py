@@ -100,3 +100,15 @@ def test_reuse_gives_identical_expert_tensors():
         assert torch.equal(q13, a.w13[e]) and torch.equal(q2, a.w2[e])
     q13, _, q2, _ = inputs.draw_expert(spec, 5, 0, shared=True)
     assert torch.equal(q13, a.ws13[0]) and torch.equal(q2, a.ws2[0])
+
+
+def test_fp4_scale_atoms_layout_and_inverse():
+    """The ABI's FP4 scale atoms: row r, 32-element run q of a 128 x 128 block at byte
+    (r % 32) * 16 + (r / 32) * 4 + q of its 512-byte atom; scale_rows undoes it."""
+    rng = np.random.default_rng(0)
+    codes = rng.integers(0, 255, (256, 12)).astype(np.uint8)   # 2 row blocks x 3 K blocks
+    at = inputs.scale_atoms(codes).numpy()
+    assert at.shape == (2, 3, 512)
+    for rb, kb, r, q in [(0, 0, 0, 0), (1, 2, 127, 3), (0, 1, 37, 2), (1, 0, 96, 1)]:
+        assert at[rb, kb, (r % 32) * 16 + (r // 32) * 4 + q] == codes[rb * 128 + r, kb * 4 + q]
+    assert np.array_equal(inputs.scale_rows(at).numpy(), codes)

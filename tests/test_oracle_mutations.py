@@ -163,6 +163,20 @@ def _e8m0_bias_128(codes):
     return _REAL["decode_e8m0"](codes) / 2.0
 
 
+def _quantise_ties_away_from_zero(x, block=128):
+    codes, sc = _REAL["quantize_e4m3_blocks"](x, block)
+    q = np.abs(np.asarray(x, np.float64) / np.repeat(sc, block, axis=1))
+    vals = om.decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    c = codes & 0x7F
+    tie = (c < 0x7E) & (q == (vals[np.minimum(c, 0x7D)] + vals[np.minimum(c, 0x7D) + 1]) / 2)
+    return np.where(tie, codes + 1, codes).astype(np.uint8), sc
+
+
+def _quantise_scale_half(x, block=128):
+    codes, sc = _REAL["quantize_e4m3_blocks"](np.asarray(x) * 2.0, block)
+    return codes, sc / 2.0
+
+
 def _router_logits_without_transpose(x, wr):
     x, wr = np.asarray(x, np.float64), np.asarray(wr, np.float64)
     return x @ wr.reshape(wr.shape[1], wr.shape[0])
@@ -170,7 +184,7 @@ def _router_logits_without_transpose(x, wr):
 
 _REAL = {n: getattr(om, n) for n in ("gate_weights", "selection_keys", "combine", "decode_e4m3",
                                       "dequantize_blocks", "decode_e2m1", "unpack_fp4",
-                                      "decode_e8m0")}
+                                      "decode_e8m0", "quantize_e4m3_blocks")}
 
 MUTATIONS = [
     ("select_topk", _topk_ties_to_higher_index),
@@ -190,6 +204,8 @@ MUTATIONS = [
     ("decode_e2m1", _e2m1_exponent_bias_0),
     ("unpack_fp4", _fp4_nibbles_swapped),
     ("decode_e8m0", _e8m0_bias_128),
+    ("quantize_e4m3_blocks", _quantise_ties_away_from_zero),
+    ("quantize_e4m3_blocks", _quantise_scale_half),
 ]
 
 

@@ -168,6 +168,32 @@ def test_table_mxfp4_helper_equals_oracle():
     assert np.array_equal(dequant_mxfp4_fast(packed, sc), oracle.dequantize_mxfp4(packed, sc))
 
 
+def test_e4m3_block_quantisation_matches_torch():
+    """Codes: torch's float8_e4m3fn conversion (round to nearest even) of x / 2^e; scales: the
+    smallest power of two that brings the block's amax to 448 or below."""
+    rng = np.random.default_rng(8)
+    x = (rng.standard_normal((64, 512)) * np.exp2(rng.integers(-20, 20, (64, 4))).repeat(128, 1))
+    x = inputs.to_bf16(x.astype(np.float32)).double().numpy()     # bf16 values, as the layer gets
+    x[0, :128] = 0.0
+    x[1, :128] = 0.0
+    x[1, 5] = -448.0 * 2.0 ** 3                                   # amax exactly 448 * 2^3
+    x[2, 128:256] = -1e-30                                        # rounds to negative zero
+    x[2, 128] = 1.0
+    codes, sc = oracle.quantize_e4m3_blocks(x)
+    e = np.log2(sc)
+    assert np.array_equal(e, np.round(e))
+    amax = np.abs(x).reshape(64, 4, 128).max(axis=2)
+    assert np.all(amax <= 448.0 * sc) and np.all((amax > 224.0 * sc) | (amax == 0))
+    assert sc[0, 0] == 1.0 and np.all(codes[0, :128] == 0)
+    assert sc[1, 0] == 8.0 and codes[1, 5] == 0xFE
+    assert np.all(codes[2, 129:256] == 0x80)
+    lib = torch.from_numpy(x / np.repeat(sc, 128, axis=1)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, lib)
+    # and the stored-input encoder of the generator agrees on power-of-two scaled data
+    q, s = inputs.to_e4m3_blocks(x.astype(np.float32), 1, 128)
+    assert np.array_equal(q.view(torch.uint8).numpy(), codes) and np.array_equal(s.numpy(), sc)
+
+
 def test_table_dequant_helper_equals_oracle():
     """The tests' table-driven block dequantisation (used on whole expert weight sets) gives
     oracle.dequantize_blocks's values bit for bit, every code and block shape included."""
