@@ -291,8 +291,10 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
-  const bool m256 = false;
-  g.mode = w4 ? kFFN2F4 : kFFN2F8;
+  // decode-sized token tiles: two 128-row weight blocks per tile (256 output columns), as
+  // d_model allows
+  const bool m256 = chunk_rows == kChunkRowsNarrow && d % 256 == 0;
+  g.mode = m256 ? (w4 ? kFFN2F4M256 : kFFN2F8M256) : (w4 ? kFFN2F4 : kFFN2F8);
   g.halves = false;
   g.gather = false;
   g.tile_tokens = chunk_rows;
