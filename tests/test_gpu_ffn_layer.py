@@ -213,6 +213,7 @@ def test_layer_tiny_config():
     (130, 128, 1, 1, 128, 0, "softmax"),          # E = 1, k = 1: a dense SwiGLU FFN
     (520, 256, 4, 2, 128, 1, "sigmoid_bias"),     # heavy groups: several 128-row chunks each
     (96, 1024, 16, 4, 256, 1, "sigmoid_bias"),    # decode-sized, two 512-row FFN2 weight tiles
+    (129, 256, 8, 4, 128, 1, "softmax"),          # smallest batch on wide (256-row) chunks
 ])
 def test_layer_custom(T, d, E, k, I, S, score):
     spec = inputs.custom_spec(T, d, E, k, I, S, score=score)

@@ -174,6 +174,33 @@ def test_permute_quantises_bf16_rows_for_low_precision_experts(T, E, k, d, weigh
     assert np.array_equal(x_perm_s.cpu().numpy().astype(np.float64), sc[rp])
 
 
+def test_quantising_permute_drops_out_of_range_pairs():
+    """Pairs with an expert index outside [0, E) are dropped by the quantising permutation as
+    by the plain one (inv_perm -1, not counted) and reported in the device status."""
+    T, E, k, d = 40, 8, 2, 256
+    idx = np.tile(np.array([0, 1]), (T, 1))
+    idx[5, 1] = 8
+    idx[9, 0] = -1
+    x = inputs.to_bf16(np.random.default_rng(3).standard_normal((T, d)).astype(np.float32))
+    cfg = moe.make_config(T, d, E, k, 128, 0, act="bf16", weight="e4m3")
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    R = T * k
+    x_perm = torch.zeros((R, d), dtype=torch.uint8, device=DEV)
+    x_perm_s = torch.zeros((R, d // 128), dtype=torch.float32, device=DEV)
+    perm_token = torch.empty(R, dtype=torch.int32, device=DEV)
+    inv_perm = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    moe.moe_permute(cfg, torch.from_numpy(idx.astype(np.int32)).to(DEV), x.to(DEV), None, x_perm,
+                    x_perm_s, perm_token, inv_perm, offsets, ws)
+    assert moe.moe_read_device_status(ws) == 5
+    ip = inv_perm.cpu().numpy()
+    assert ip[5, 1] == -1 and ip[9, 0] == -1 and offsets.cpu().numpy()[-1] == R - 2
+    codes, sc = oracle.quantize_e4m3_blocks(x.double().numpy())
+    pt = perm_token.cpu().numpy()[: R - 2]
+    assert np.array_equal(x_perm.cpu().numpy()[: R - 2], codes[pt])
+    assert np.array_equal(x_perm_s.cpu().numpy()[: R - 2].astype(np.float64), sc[pt])
+
+
 def test_permute_fp8_rows_and_scales():
     T, E, k, d = 300, 32, 4, 256
     rng = np.random.default_rng(9)
@@ -221,7 +248,8 @@ def _check_fp8_layer(wl, rows=None, routing=None):
 
 
 @pytest.mark.parametrize("T,d,E,k,I,S", [(70, 256, 16, 4, 256, 1), (300, 384, 8, 2, 128, 2),
-                                         (1, 128, 4, 1, 128, 1)])
+                                         (1, 128, 4, 1, 128, 1),
+                                         (129, 512, 8, 4, 256, 1)])   # smallest wide-tile batch
 @pytest.mark.parametrize("weight", ["e4m3", "e2m1"])
 def test_layer_fp8_custom(T, d, E, k, I, S, weight):
     spec = inputs.custom_spec(T, d, E, k, I, S, act="e4m3", weight=weight)
