@@ -189,6 +189,11 @@ class ClockSampler:
 # algorithmic work
 # ---------------------------------------------------------------------------
 
+def _e4m3(dtype):
+    """e4m3 storage, with power-of-two ("e4m3") or any fp32 ("e4m3_fs") block scales."""
+    return dtype in ("e4m3", "e4m3_fs")
+
+
 def work_model(spec, offsets):
     """Algorithmic bytes / flops of the layer and of its two expert GEMM launches.
 
@@ -199,8 +204,8 @@ def work_model(spec, offsets):
     """
     T, d, E, k, I, S = spec.T, spec.d_model, spec.E, spec.top_k, spec.d_ff, spec.n_shared
     # weight bytes per element: MXFP4 = half a byte + one E8M0 byte per 32 elements
-    wb = {"e4m3": 1.0, "e2m1": 0.5 + 1.0 / 32}.get(spec.weight, 2.0)
-    ab = 1 if spec.act == "e4m3" else 2
+    wb = {"e4m3": 1.0, "e4m3_fs": 1.0, "e2m1": 0.5 + 1.0 / 32}.get(spec.weight, 2.0)
+    ab = 1 if _e4m3(spec.act) else 2
     sizes = np.diff(offsets)
     touched = int((sizes > 0).sum())
     R = T * k
@@ -226,8 +231,8 @@ def small_stage_bytes(spec):
     """Algorithmic HBM bytes of the bandwidth-bound stages around the expert GEMMs (reads +
     writes each stage must make at least once)."""
     T, d, E, k, S = spec.T, spec.d_model, spec.E, spec.top_k, spec.n_shared
-    ab = 1 if spec.act == "e4m3" else 2
-    xs = 4 * (d // 128) if spec.act == "e4m3" else 0          # per-row activation scales
+    ab = 1 if _e4m3(spec.act) else 2
+    xs = 4 * (d // 128) if _e4m3(spec.act) else 0          # per-row activation scales
     ob = 4 if spec.out == "f32" else 2
     R = T * k
     return {
@@ -565,17 +570,25 @@ def time_graph(moe, layer, x, xs, y, idx, gw, K, W, stream, dev, barrier, max_ov
 
 
 def launches_per_step(spec):
-    """Kernels one ``moe_layer_forward`` launches: router GEMM, route, permute (count and
-    gather for T <= 256, else count, rank and gather), plan, FFN1, FFN2, combine; the
-    f32 family adds its bf16 conversions, the FP8 family its scale preparation and the
-    gather of the permuted rows' scales."""
-    n = 1 + 1 + (2 if spec.T <= 256 else 3) + 1 + 2 + 1
+    """Kernels one ``moe_layer_forward`` launches: router GEMM, route, permute (count, then
+    rank for T > 256, then the row copy -- none when the first GEMM gathers e4m3 rows on
+    wide tiles, T > 128), plan, FFN1, FFN2, combine; the f32 family adds its bf16
+    conversions, e4m3 activations their scale preparation (and, on decode-sized tiles with
+    power-of-two scales, the permuted rows' scale gather), e4m3 weights with power-of-two
+    scales their UE8M0 conversion."""
+    wide = spec.T > 128
+    e4m3_tok = _e4m3(spec.act) or spec.weight in ("e4m3", "e2m1")
+    gather = e4m3_tok and wide and spec.weight != "e4m3_fs"
+    quant = spec.act == "bf16" and spec.weight in ("e4m3", "e2m1")
+    n = 1 + 1 + 1 + (1 if spec.T > 256 else 0) + (0 if gather and not quant else 1) + 1 + 2 + 1
     if spec.act == "f32":
         n += 4 + (2 if spec.n_shared else 0)
-    if spec.act == "e4m3":
-        n += 1 + 1                     # activation scale preparation, permuted-row scales
+    if _e4m3(spec.act):
+        n += 1                                  # activation scale preparation
+        if spec.act == "e4m3" and not gather:
+            n += 1                              # permuted rows' UE8M0 scale factors
     if spec.weight == "e4m3":
-        n += 2 + (2 if spec.n_shared else 0)   # weight block scales -> UE8M0
+        n += 2 + (2 if spec.n_shared else 0)    # weight block scales -> UE8M0
     return n
 
 
@@ -669,7 +682,7 @@ def run_ours(args):
         dom = "ffn1"
         achieved = wm["ffn1_flops"] / (stage_ms["ffn1"] * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        if spec.weight == "e4m3":
+        if _e4m3(spec.weight):
             fp8 = load_fp8_peak()
             if fp8 is not None:
                 peak, peak_src = fp8, "measured e4m3 sustained (profiles/peaks.json)"
@@ -679,7 +692,7 @@ def run_ours(args):
         unit = "TFLOP/s"
         units_note = "2 * (T*k + S*T) * 2I * d"
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    if spec.weight == "e4m3":
+    if _e4m3(spec.weight):
         tensor_peak = load_fp8_peak() or 2.0 * tensor_peak
     ffn_bound_ms = per_expert_bound_ms(wm, tensor_peak, peaks["hbm_gbs"])
     tokens = spec.T * world
@@ -688,7 +701,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": {"e4m3": "e4m3", "e2m1": "e2m1 x e4m3"}.get(spec.weight, "bf16"),
+        "dtype": {"e4m3": "e4m3", "e4m3_fs": "e4m3 (fp32 block scales)",
+                  "e2m1": "e2m1 x e4m3"}.get(spec.weight, "bf16"),
         "data": "synthetic",
         "config": {"workload": name if not args.experts else
                    f"{name} with E={spec.E}, T={spec.T} (profiling case)",
@@ -698,7 +712,8 @@ def run_ours(args):
                    "l2": "inputs larger than L2: each step streams "
                          f"{wm['layer_weight_bytes'] / 1e9:.1f} GB of expert weights"},
         "roofline": {"bound": bound,
-                     "kernel": f"{dom} (grouped_gemm_kernel<{ {'e4m3': 3, 'e2m1': 7}.get(spec.weight, 1)}>)",
+                     "kernel": f"{dom} (" + ("grouped_gemm_fs_kernel<11>" if spec.weight == "e4m3_fs" else
+                                             f"grouped_gemm_kernel<{ {'e4m3': 3, 'e2m1': 7}.get(spec.weight, 1)}>") + ")",
                      "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": unit,
                      "frac": achieved / peak, "traffic": read_traffic(f"ffn1_{name}"),
                      "units": units_note},
@@ -758,7 +773,7 @@ def run_stages(args):
     bias = None if spec.score != "sigmoid_bias" else 0.1 * torch.rand(E, generator=g, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     gw = torch.empty((T, k), dtype=torch.float32, device=dev)
-    fp8 = spec.act == "e4m3"
+    fp8 = _e4m3(spec.act)
     x = torch.randn((T, d), generator=g, device=dev).to(torch.bfloat16)
     xs = xps = None
     if fp8:

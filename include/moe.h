@@ -98,7 +98,15 @@ typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_BIAS = 1 } moe_score_fn;
  * rows x 128 K-elements, [rows/128][K/128][512]: inside an atom the scale of row r (0..127)
  * and 32-element run q (0..3) sits at byte (r % 32) * 16 + (r / 32) * 4 + q -- the layout
  * the tensor cores' scale-factor copy takes, so the kernels copy atoms without reshuffling. */
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2, MOE_E2M1 = 3 } moe_dtype;
+/* MOE_E4M3_FP32_SCALE: e4m3 values whose fp32 block scales (1x128 for activations, 128x128
+ * for weights, as for MOE_E4M3) may be any positive finite value, not only powers of two.
+ * The expert GEMMs then multiply without block scaling and fold each 128-K block's
+ * s_weight * s_activation into fp32 accumulators (exact up to fp32 rounding), on 32-token
+ * tiles: slower than MOE_E4M3, whose power-of-two scales the tensor cores apply directly.
+ * Activations and weights both take this dtype.  The router takes x = code x scale as a
+ * bf16 part plus its bf16 remainder (two router GEMMs, summed with the split-K partials):
+ * x to ~2^-17 relative, where a single bf16 rounding would move the logits by ~2^-9. */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2, MOE_E2M1 = 3, MOE_E4M3_FP32_SCALE = 4 } moe_dtype;
 
 /* The layer's sizes: T tokens x d_model activations, E routed experts, top_k,
  * expert intermediate size d_ff (I), n_shared always-on shared experts of

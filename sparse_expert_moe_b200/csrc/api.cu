@@ -25,15 +25,26 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 // The expert GEMMs take e4m3 token rows: e4m3 activations, or bf16 activations quantised
 // in the permutation because the expert weights are e4m3 or FP4.
 inline bool tok_e4m3(const moe_config& c) {
-  return c.act == MOE_E4M3 || c.weight == MOE_E4M3 || c.weight == MOE_E2M1;
+  return c.act == MOE_E4M3 || c.weight == MOE_E4M3 || c.weight == MOE_E2M1 ||
+         c.act == MOE_E4M3_FP32_SCALE;
 }
+// e4m3 operands with arbitrary fp32 block scales (exact per-K-block rescale)
+inline bool fp32_scaled(const moe_config& c) { return c.weight == MOE_E4M3_FP32_SCALE; }
+
+// K splits of the router GEMM, and the partial logit arrays the route kernel sums: with
+// fp32-scaled activations the router runs on x's bf16 part and on its bf16 remainder (two
+// sets of splits, at most 32 partials in all).
+inline int router_k_splits(const moe_config& c) {
+  return router_splits(c.T, c.E, c.d_model, fp32_scaled(c) ? 16 : 32);
+}
+inline int router_parts(const moe_config& c) { return (fp32_scaled(c) ? 2 : 1) * router_k_splits(c); }
 inline bool quant_in_permute(const moe_config& c) { return c.act == MOE_BF16 && tok_e4m3(c); }
 
 // Byte offsets of every workspace region for one configuration.
 struct Layout {
   size_t logits, topk_idx, topk_w, offsets, chunk_counts, perm_token, inv_perm, x_perm, chunks,
       grp_cp, h,
-      y_rows, x_bf16, wr_bf16, w13_bf16, w2_bf16, a_bf16, x_sf, x_perm_sf, h_sf, a_sf, wsf13, wsf2,
+      y_rows, x_bf16, x_lo, wr_bf16, w13_bf16, w2_bf16, a_bf16, x_sf, x_perm_sf, h_sf, a_sf, wsf13, wsf2,
       total;
   int64_t R, rows_all, n_chunk_max;
 
@@ -52,7 +63,7 @@ struct Layout {
       o = align_up(o + bytes);
       return at;
     };
-    logits = take(sizeof(float) * router_splits(T, E, d) * T * E);
+    logits = take(sizeof(float) * router_parts(c) * T * E);
     topk_idx = take(sizeof(int32_t) * R);
     topk_w = take(sizeof(float) * R);
     offsets = take(sizeof(int32_t) * (E + 1));
@@ -65,6 +76,7 @@ struct Layout {
     h = take(2 * rows_all * I);
     y_rows = take(2 * rows_all * d);
     x_bf16 = take(f32 || fp8 ? 2 * T * d : 0);   // q8: the quantised x [T, d] e4m3
+    x_lo = take(fp32_scaled(c) ? 2 * T * d : 0);  // bf16 remainder of fp32-scaled x
     (void)q8;
     wr_bf16 = take(f32 ? 2 * E * d : 0);
     w13_bf16 = take(f32 ? 2 * (E + S) * 2 * I * d : 0);
@@ -109,7 +121,8 @@ moe_status check_config(const moe_config* c) {
   const bool fam_w4a8 = c->act == MOE_E4M3 && c->weight == MOE_E2M1;
   // bf16 activations into e4m3 or FP4 experts: quantised to e4m3 in the permutation
   const bool fam_q8 = c->act == MOE_BF16 && (c->weight == MOE_E4M3 || c->weight == MOE_E2M1);
-  if (!(fam_bf16 || fam_f32 || fam_fp8 || fam_w4a8 || fam_q8)) return MOE_ERR_UNSUPPORTED;
+  const bool fam_fs = c->act == MOE_E4M3_FP32_SCALE && c->weight == MOE_E4M3_FP32_SCALE;
+  if (!(fam_bf16 || fam_f32 || fam_fp8 || fam_w4a8 || fam_q8 || fam_fs)) return MOE_ERR_UNSUPPORTED;
   if (c->out != MOE_BF16 && c->out != MOE_F32) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -327,6 +340,86 @@ moe_status run_ffn_fp8(const moe_config& c, const Layout& L, void* ws, const Fp8
 // The two expert GEMMs over a chunk list already planned into the workspace.
 // seg 0: routed (a0 rows, w13_0 / w2_0 with G0 groups); seg 1: shared (a1 rows,
 // w13_1 / w2_1 with S groups) or absent.  h and y have rows_all rows.
+// The e4m3 expert GEMMs with arbitrary fp32 block scales over a chunk list of 32-row chunks
+// planned into the workspace: seg0 the routed rows, seg1 the shared experts (groups = 0:
+// absent).  a_scale: fp32 [a_rows][d/128]; w13_s / w2_s: fp32 128x128 block scales.  h
+// (e4m3, power-of-two 1x128 scales as UE8M0 words) lives in the workspace.
+struct FsSeg {
+  const void* a;
+  const float* a_scale;
+  int64_t a_rows;
+  const void* w13;
+  const void* w2;
+  const float* w13_s;
+  const float* w2_s;
+  int64_t groups;
+};
+
+moe_status run_ffn_fs(const moe_config& c, const Layout& L, void* ws, const FsSeg& s0,
+                      const FsSeg& s1, int64_t rows_all, void* y, cudaStream_t s,
+                      cudaEvent_t* ev = nullptr) {
+  const int64_t d = c.d_model, I = c.d_ff;
+  void* h = at<void>(ws, L.h);
+  uint32_t* h_sf = at<uint32_t>(ws, L.h_sf);
+  const FsSeg* seg[2] = {&s0, s1.groups > 0 ? &s1 : &s0};
+  GemmLaunch g{};
+  g.chunks = at<Chunk>(ws, L.chunks);
+  g.n_chunks = at<int32_t>(ws, kHdrNChunks * sizeof(int));
+  g.grp_cp = at<int32_t>(ws, L.grp_cp);
+  g.n_grp = at<int32_t>(ws, kHdrNGroups * sizeof(int));
+  g.status = status_word(ws);
+  g.num_sms = num_sms();
+
+  g.mode = kFFN1X;
+  for (int i = 0; i < 2; ++i) {
+    const FsSeg& q = *seg[i];
+    if (!make_tmap_u8(&g.wmap[i], q.w13, q.groups * 2 * I, d, 128) ||
+        !make_tok_maps(g.tmap[i], q.a, q.a_rows, d, true))
+      return MOE_ERR_CUDA;
+    g.fs_a[i] = q.a_scale;
+    g.fs_w[i] = q.w13_s;
+  }
+  g.fs_a_ld = static_cast<int>(d / 128);
+  g.n_mblk = static_cast<int>(I / 128);
+  g.k_blocks = static_cast<int>(d / 128);
+  g.w_rows_per_group = static_cast<int>(2 * I);
+  g.wsf_rb_per_group = static_cast<int>(2 * I / 128);
+  g.up_offset = static_cast<int>(I);
+  g.m_valid = static_cast<int>(I);
+  g.out = h;
+  g.ld_out = static_cast<int>(I);
+  g.out_sf = h_sf;
+  g.ld_out_sf = static_cast<int>(rows_all);
+  moe_status st = cuda_status(launch_gemm(g, s));
+  if (st != MOE_OK) return st;
+  if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
+
+  g.mode = kFFN2X;
+  if (!make_tok_maps(g.tmap[0], h, rows_all, I, true)) return MOE_ERR_CUDA;
+  copy_maps(g.tmap[1], g.tmap[0]);
+  for (int i = 0; i < 2; ++i) {
+    const FsSeg& q = *seg[i];
+    if (!make_tmap_u8(&g.wmap[i], q.w2, q.groups * d, I, 128)) return MOE_ERR_CUDA;
+    g.fs_w[i] = q.w2_s;
+    g.tsf[i] = h_sf;
+    g.tsf_ld[i] = static_cast<int>(rows_all);
+    g.tsf_rows[i] = static_cast<int>(rows_all);
+  }
+  g.n_mblk = static_cast<int>(d / 128);
+  g.k_blocks = static_cast<int>(I / 128);
+  g.w_rows_per_group = static_cast<int>(d);
+  g.wsf_rb_per_group = static_cast<int>(d / 128);
+  g.up_offset = 0;
+  g.m_valid = static_cast<int>(d);
+  g.out = y;
+  g.ld_out = static_cast<int>(d);
+  g.out_sf = nullptr;
+  st = cuda_status(launch_gemm(g, s));
+  if (st != MOE_OK) return st;
+  if (ev) st = cuda_status(cudaEventRecord(ev[1], s));
+  return st;
+}
+
 moe_status run_ffn(const moe_config& c, const Layout& L, void* ws, const void* a0, int64_t a0_rows,
                    const void* w13_0, const void* w2_0, int64_t G0, const void* a1, int64_t a1_rows,
                    const void* w13_1, const void* w2_1, int64_t S, int64_t rows_all, void* y,
@@ -444,7 +537,7 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
         nullptr, nullptr, perm_token, inv_perm, group_offsets, at<int32_t>(ws, L.chunk_counts),
         at<unsigned>(ws, kHdrPermuteDone * sizeof(int)), status_word(ws), stream));
   }
-  const bool fp8 = cfg->act == MOE_E4M3;
+  const bool fp8 = cfg->act == MOE_E4M3 || cfg->act == MOE_E4M3_FP32_SCALE;
   if (fp8 && cfg->T > 0 && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
   const int elem = cfg->act == MOE_F32 ? 4 : (fp8 ? 1 : 2);
   return cuda_status(launch_permute(topk_idx, cfg->T, cfg->E, cfg->top_k, x, cfg->d_model * elem,
@@ -492,6 +585,17 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
     a_b = at<void>(ws, L.a_bf16);
     w13_b = at<void>(ws, L.w13_bf16);
     w2_b = at<void>(ws, L.w2_bf16);
+  }
+  if (fp32_scaled(*cfg)) {   // e4m3 rows and weights with arbitrary fp32 block scales
+    if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
+    st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRowsNarrow,
+                                 at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
+                                 at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
+                                 status_word(ws), stream));
+    if (st != MOE_OK) return st;
+    const FsSeg s0{a, a_scale, n_rows, w13, w2, static_cast<const float*>(w13_s),
+                   static_cast<const float*>(w2_s), n_groups};
+    return run_ffn_fs(*cfg, L, ws, s0, FsSeg{}, n_rows, y, stream);
   }
   if (tok_e4m3(*cfg)) {   // e4m3 token rows (as moe_permute gives them for e4m3 / FP4 experts)
     if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
@@ -572,6 +676,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
     return MOE_ERR_INVALID_ARG;
   const bool fp8 = tok_e4m3(c);            // e4m3 token operand of the expert GEMMs
   const bool q8 = quant_in_permute(c);     // ... quantised from bf16 x in the permutation
+  const bool fs = fp32_scaled(c);          // ... with arbitrary fp32 block scales
   const bool w4 = c.weight == MOE_E2M1;
   if (fp8 && ((!q8 && !x_scale) || !wts->w13_s || !wts->w2_s ||
               (c.n_shared > 0 && (!wts->ws13_s || !wts->ws2_s))))
@@ -625,11 +730,12 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   const size_t n13 = static_cast<size_t>(2 * I / 128) * (d / 128);
   const size_t n2 = static_cast<size_t>(d / 128) * (I / 128);
   if (fp8) {
-    if (!q8)
+    if (!q8)   // fp32-scaled rows: no UE8M0 factors (no power-of-two check), a bf16 remainder
       st = cuda_status(launch_act_prep_fp8(static_cast<const uint8_t*>(x), x_scale, c.T,
-                                           static_cast<int>(d), at<void>(ws, L.x_bf16), x_sf,
-                                           status, s));
-    if (!w4) {   // e4m3 weights: fp32 block scales -> UE8M0 scale factors
+                                           static_cast<int>(d), at<void>(ws, L.x_bf16),
+                                           fs ? nullptr : x_sf, status, s,
+                                           fs ? at<void>(ws, L.x_lo) : nullptr));
+    if (c.weight == MOE_E4M3) {   // power-of-two fp32 block scales -> UE8M0 scale factors
       auto wsf = [&](const void* src, size_t n, uint4* dst) {
         return cuda_status(launch_weight_sf(static_cast<const float*>(src), n, dst, status, s));
       };
@@ -655,7 +761,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
     g.router_T = static_cast<int>(T);
     g.n_mblk = static_cast<int>((E + 127) / 128);
     g.k_blocks = static_cast<int>(d / 64);
-    g.k_splits = router_splits(T, E, d);
+    g.k_splits = router_k_splits(c);
     g.split_stride = static_cast<long long>(T) * E;
     g.m_valid = static_cast<int>(E);
     g.out = logits;
@@ -664,6 +770,13 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
     g.num_sms = num_sms();
     st = cuda_status(launch_gemm(g, s));
     if (st != MOE_OK) return st;
+    if (fs) {   // the bf16 remainder of x into the next set of partial logits
+      if (!make_tok_maps(g.tmap[0], at<void>(ws, L.x_lo), T, d, false)) return MOE_ERR_CUDA;
+      copy_maps(g.tmap[1], g.tmap[0]);
+      g.out = logits + static_cast<size_t>(g.k_splits) * T * E;
+      st = cuda_status(launch_gemm(g, s));
+      if (st != MOE_OK) return st;
+    }
   }
   if ((st = mark(1)) != MOE_OK) return st;
 
@@ -671,7 +784,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
   float* gate = topk_w_out ? topk_w_out : at<float>(ws, L.topk_w);
   const float* bias = c.score == MOE_SCORE_SIGMOID_BIAS ? wts->sel_bias : nullptr;
-  st = cuda_status(launch_route(logits, router_splits(T, E, d), static_cast<long long>(T) * E, bias,
+  st = cuda_status(launch_route(logits, router_parts(c), static_cast<long long>(T) * E, bias,
                                 c.T, c.E, c.top_k, c.score, idx, gate, s));
   if (st != MOE_OK) return st;
   if ((st = mark(2)) != MOE_OK) return st;
@@ -682,7 +795,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   // here; otherwise the rows are copied into x_perm (bf16 rows, or e4m3 rows + scale
   // factors).  bf16 rows keep the copy: measured on the R1 prefill layer, the first GEMM
   // fed by TMA from x_perm is faster than with gathered rows by more than the copy costs.
-  const int chunk_rows = fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T);
+  const int chunk_rows = fs ? kChunkRowsNarrow : (fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T));
   const bool gather = fp8 && chunk_rows != kChunkRowsNarrow;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm_token = at<int32_t>(ws, L.perm_token);
@@ -704,6 +817,11 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   } else if (gather) {
     st = cuda_status(launch_permute_index(idx, c.T, c.E, c.top_k, perm_token, inv_perm, offsets,
                                           counts, ticket, status, s));
+  } else if (fs) {   // e4m3 rows with their fp32 scales, [R][d/128]
+    st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(d), x_scale,
+                                    static_cast<int>(d / 128), x_perm,
+                                    reinterpret_cast<float*>(x_perm_sf), perm_token, inv_perm,
+                                    offsets, counts, ticket, status, s));
   } else {
     st = cuda_status(launch_permute(idx, c.T, c.E, c.top_k, x_b, static_cast<int>(fp8 ? d : d * 2),
                                     nullptr, 0, x_perm, nullptr, perm_token, inv_perm, offsets,
@@ -724,7 +842,13 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   if (st != MOE_OK) return st;
   if ((st = mark(4)) != MOE_OK) return st;
   void* y_rows = at<void>(ws, L.y_rows);
-  if (fp8) {
+  if (fs) {
+    const FsSeg s0{x_perm, reinterpret_cast<const float*>(x_perm_sf), R, w13_b, w2_b,
+                   static_cast<const float*>(wts->w13_s), static_cast<const float*>(wts->w2_s), E};
+    const FsSeg s1{x_b, x_scale, T, ws13_b, ws2_b, static_cast<const float*>(wts->ws13_s),
+                   static_cast<const float*>(wts->ws2_s), S};
+    st = run_ffn_fs(c, L, ws, s0, s1, L.rows_all, y_rows, s, ev ? ev + 5 : nullptr);
+  } else if (fp8) {
     Fp8Seg s0{x_perm, x_perm_sf, R, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E, nullptr};
     if (gather) s0 = Fp8Seg{x_tok, x_sf, T, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E, perm_token};
     Fp8Seg s1{x_tok, x_sf, T, ws13_b, ws2_b, nullptr, nullptr, nullptr, nullptr, S, nullptr};

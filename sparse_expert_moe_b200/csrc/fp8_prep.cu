@@ -26,10 +26,13 @@ __device__ __forceinline__ uint32_t ue8m0x4(float s, int* status) {
   return 0x01010101u * e;
 }
 
-// One thread per 16 activation bytes (16 e4m3 values, one 1x128 scale block).
+// One thread per 16 activation bytes (16 e4m3 values, one 1x128 scale block).  x_lo
+// (optional): v - bf16(v) rounded to bf16, so that x_bf16 + x_lo carries v = code x scale to
+// ~2^-17 relative when the scale is not a power of two (x_bf16 alone is then rounded).
 __global__ void act_prep_fp8_kernel(const uint4* __restrict__ x, const float* __restrict__ x_scale,
                                     int T, int d, uint4* __restrict__ x_bf16,
-                                    uint32_t* __restrict__ x_sf, int* status) {
+                                    uint4* __restrict__ x_lo, uint32_t* __restrict__ x_sf,
+                                    int* status) {
   const int vec_per_row = d / 16;
   const size_t n = static_cast<size_t>(T) * vec_per_row;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -41,16 +44,24 @@ __global__ void act_prep_fp8_kernel(const uint4* __restrict__ x, const float* __
     if (x_bf16) {
       const uint4 q = x[i];
       const __nv_fp8x2_storage_t* p = reinterpret_cast<const __nv_fp8x2_storage_t*>(&q);
-      uint4 o[2];
+      uint4 o[2], lo[2];
       __nv_bfloat162* ob = reinterpret_cast<__nv_bfloat162*>(o);
+      __nv_bfloat162* ol = reinterpret_cast<__nv_bfloat162*>(lo);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(p[j], __NV_E4M3);
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-        ob[j] = __floats2bfloat162_rn(f.x * s, f.y * s);
+        const float2 v = make_float2(f.x * s, f.y * s);
+        ob[j] = __floats2bfloat162_rn(v.x, v.y);
+        const float2 h = __bfloat1622float2(ob[j]);
+        ol[j] = __floats2bfloat162_rn(v.x - h.x, v.y - h.y);
       }
       x_bf16[2 * i] = o[0];
       x_bf16[2 * i + 1] = o[1];
+      if (x_lo) {
+        x_lo[2 * i] = lo[0];
+        x_lo[2 * i + 1] = lo[1];
+      }
     }
     if (x_sf && (v % 8) == 0) x_sf[static_cast<size_t>(kb) * T + t] = ue8m0x4(s, status);
   }
@@ -88,11 +99,12 @@ unsigned grid_for(size_t n, int threads) {
 }  // namespace
 
 cudaError_t launch_act_prep_fp8(const uint8_t* x, const float* x_scale, int T, int d, void* x_bf16,
-                                uint32_t* x_sf, int* status, cudaStream_t s) {
+                                uint32_t* x_sf, int* status, cudaStream_t s, void* x_lo) {
   if (T == 0) return cudaSuccess;
   const size_t n = static_cast<size_t>(T) * (d / 16);
   act_prep_fp8_kernel<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), x_scale, T,
-                                                       d, static_cast<uint4*>(x_bf16), x_sf, status);
+                                                       d, static_cast<uint4*>(x_bf16),
+                                                       static_cast<uint4*>(x_lo), x_sf, status);
   return cudaGetLastError();
 }
 

@@ -88,6 +88,12 @@ struct DevParams {
   const uint8_t* gsrc[2];
   const int32_t* gidx[2];
   int g_ld;
+  // fp32-scale modes (kFFN1X / kFFN2X): token scales fp32 [rows][fs_a_ld] per segment
+  // (kFFN1X; kFFN2X reads h's UE8M0 words through tsf), weight scales fp32
+  // [groups][row blocks][k blocks] per segment
+  const float* fs_a[2];
+  int fs_a_ld;
+  const float* fs_w[2];
 };
 
 // NTW: token-tile width of the bf16 expert GEMMs.  128 by default -- half of a 256-row
@@ -751,6 +757,330 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW, GATHER>::kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+
+// ---------------------------------------------------------------- fp32 block scales
+// e4m3 expert GEMMs whose block scales are arbitrary positive fp32 values (not powers of
+// two, which the tensor cores' UE8M0 scale factors cannot hold).  The MMAs run without
+// block scaling (kind::f8f6f4); every 128-K block accumulates into its own TMEM buffer
+// (two, alternating), and the epilogue warps fold it into fp32 register accumulators as
+//   acc[r][n] += (s_w[block of r][kb] * s_a[n][kb]) * partial_kb[r][n]
+// -- the block-scaled product summed exactly as its definition states, in fp32.  Tiles are
+// 32 tokens wide (the accumulators of a tile live in registers), 128 weight rows (two
+// tiles, gate and up, for the first GEMM).
+//   warp 0  TMA producer; warp 1  MMA issuer (also moves each block's scales from the stage
+//   to a per-buffer slot the epilogue reads); warps 2-5  epilogue; warp 6  scale warp
+//   (cp.async of the stage's raw token and weight scales).
+template <int MODE>
+struct CfgFS {
+  static constexpr bool kGLU = MODE == kFFN1X;
+  static constexpr int kATiles = kGLU ? 2 : 1;
+  static constexpr int kNT = kChunkRowsNarrow;                    // 32 tokens
+  static constexpr uint32_t kBBytes = kNT * kRowBytes;
+  static constexpr uint32_t kRawBytes = 1024;                     // [32] token + [2] weight scales
+  static constexpr uint32_t kStageBytes = kATiles * kABytes + kBBytes + kRawBytes;
+  static constexpr int kStages = (192u * 1024u) / kStageBytes > 10 ? 10 : (192u * 1024u) / kStageBytes;
+  static constexpr uint32_t kPCols = kATiles * kNT;               // per partial buffer
+  static constexpr uint32_t kTmemCols = 2 * kPCols <= 64 ? 64 : 128;
+  static constexpr int kThreads = 224;
+  static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;
+  static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;
+  static constexpr uint32_t kRedBytes = 2 * 4 * 128 * 4;
+  static constexpr uint32_t kPScaleBytes = 2 * 64 * 4;            // [2 buffers][32 token + 2 weight]
+  static constexpr uint32_t kFixedBytes =
+      1024 + kStagingBytes + kGrpBytes + kRedBytes + kPScaleBytes + 1024;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kFixedBytes;
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
+    grouped_gemm_fs_kernel(const __grid_constant__ DevParams p) {
+  using C = CfgFS<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty_bar = full_bar + C::kStages;
+  uint64_t* pfull = empty_bar + C::kStages;                      // [2] partial buffer written
+  uint64_t* pempty = pfull + 2;                                  // [2] partial buffer read
+  uint64_t* red_bar = pempty + 2;                                // [2] amax exchange
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* staging = smem + C::kStages * C::kStageBytes + 1024;
+  int32_t* grp_cp = reinterpret_cast<int32_t*>(staging + C::kStagingBytes);
+  uint32_t* red = reinterpret_cast<uint32_t*>(staging + C::kStagingBytes + C::kGrpBytes);
+  float* pscale = reinterpret_cast<float*>(staging + C::kStagingBytes + C::kGrpBytes + C::kRedBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full_bar[i], 1 + 32);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&pfull[i], 2);        // the MMAs' commit + the scales' copy
+      mbar_init(&pempty[i], 4);       // one arrival per epilogue warp
+      mbar_init(&red_bar[i], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.wmap[0]);
+    tma_prefetch_desc(&p.tmap[0][0]);
+  }
+  const int n_grp = *p.n_grp;
+  for (int i = threadIdx.x; i < 2 * (n_grp + 1); i += blockDim.x) grp_cp[i] = p.grp_cp[i];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int n_tiles = *p.n_chunks * p.n_mblk;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+        const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
+        if (c.nrows <= 0) continue;
+        const int a_row = c.group * p.w_rows_per_group + tc.mb * kBM;
+        const int n_pad = (c.nrows + 15) & ~15;
+        const int tok_row = MODE == kFFN2X ? c.o_row : c.b_row;
+        const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;
+        const CUtensorMap* wm = &p.wmap[c.seg];
+        for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = tiles + stage * C::kStageBytes;
+          const int kx = kb * 128;
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          tma_load_2d(st, wm, &full_bar[stage], kx, a_row);
+          if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[stage], kx, a_row + p.up_offset);
+          uint8_t* bt = st + C::kATiles * kABytes;
+          for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
+            const int rows = 128 >> bi;
+            while (n_pad - off >= rows) {
+              tma_load_2d(bt + off * kRowBytes, &p.tmap[c.seg][bi], &full_bar[stage], kx, tok_row + off);
+              off += rows;
+            }
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t kc = 0;                 // K blocks issued so far (partial buffer kc % 2)
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+        const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
+        if (c.nrows <= 0) continue;
+        const int n_pad = (c.nrows + 15) & ~15;
+        const uint32_t idesc = idesc_e4m3_f32(kBM, n_pad);
+        for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++kc) {
+          const uint32_t b = kc & 1u;
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status) ||
+              !mbar_wait(&pempty[b], ((kc >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          fence_proxy_async_smem();    // the scale warp's cp.async rows before any async read
+          const uint8_t* st = tiles + stage * C::kStageBytes;
+          const uint8_t* raw = st + C::kATiles * kABytes + C::kBBytes;
+          float* ps = pscale + b * 64;
+          // this K block's scales to the buffer's slot: token n's (fp32, or h's UE8M0 word
+          // -> 2^(code - 127)) and each weight tile's fp32 block scale
+          for (int n = 0; n < c.nrows; ++n) {
+            if (MODE == kFFN2X) {
+              const uint32_t code = reinterpret_cast<const uint32_t*>(raw)[n] & 0xFFu;
+              ps[n] = code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
+            } else {
+              ps[n] = reinterpret_cast<const float*>(raw)[n];
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < C::kATiles; ++j) ps[32 + j] = reinterpret_cast<const float*>(raw + 128)[j];
+          const uint32_t sa = smem_u32(st), sb = sa + C::kATiles * kABytes;
+          const uint32_t d0 = tmem_base + b * C::kPCols;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = umma_desc_sw128(sb + kk * 32);
+#pragma unroll
+            for (int j = 0; j < C::kATiles; ++j)
+              umma_e4m3(d0 + j * C::kNT, umma_desc_sw128(sa + j * kABytes + kk * 32), bdesc, idesc,
+                        kk ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);   // the stage's operands and raw scales are consumed
+          umma_commit(&pfull[b]);           // the partial sums are in TMEM
+          mbar_arrive(&pfull[b]);           // the scales are in their slot
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int sub = warp & 3;
+    const int m_local = sub * 32 + lane;      // weight row inside the tile
+    uint32_t kc = 0;
+    uint32_t rbuf = 0, rpar = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+      const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
+      if (c.nrows <= 0) continue;
+      float acc[C::kATiles][32];
+#pragma unroll
+      for (int j = 0; j < C::kATiles; ++j)
+#pragma unroll
+        for (int n = 0; n < 32; ++n) acc[j][n] = 0.f;
+      for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++kc) {
+        const uint32_t b = kc & 1u;
+        const bool w = mbar_wait(&pfull[b], (kc >> 1) & 1u, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float* ps = pscale + b * 64;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::kPCols;
+#pragma unroll
+        for (int j = 0; j < C::kATiles; ++j) {
+          float v0[16], v1[16];
+          tmem_ld16x2(tb + j * C::kNT, tb + j * C::kNT + 16, v0, v1);
+          const float sw = ps[32 + j];
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            acc[j][n] = fmaf(sw * ps[n], v0[n], acc[j][n]);
+            acc[j][16 + n] = fmaf(sw * ps[16 + n], v1[n], acc[j][16 + n]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pempty[b]);
+      }
+      if (!ok) break;
+      const int mb = tc.mb;
+      if (MODE == kFFN1X) {
+        // SwiGLU, then h requantised to e4m3 with one power-of-two scale per token per 128 h
+        // columns, exchanged between the four epilogue warps (as the block-scaled path does)
+        float h[32];
+        uint32_t* redt = red + rbuf * (4 * 128);
+#pragma unroll
+        for (int n = 0; n < 32; ++n) {
+          h[n] = acc[0][n] / (1.0f + __expf(-acc[0][n])) * acc[1][n];
+          const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h[n])));
+          if (lane == 0) redt[sub * 128 + n] = wmax;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_bar[rbuf]);
+        const bool rok = mbar_wait(&red_bar[rbuf], (rpar >> rbuf) & 1u, abort_flag, p.status);
+        rpar ^= 1u << rbuf;
+        if (!__all_sync(0xffffffffu, rok)) break;
+#pragma unroll
+        for (int n0 = 0; n0 < 32; n0 += 16) {
+          uint8_t q[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int n = n0 + i;
+            const uint32_t amax = max(max(redt[n], redt[128 + n]), max(redt[256 + n], redt[384 + n]));
+            const int e = e4m3_scale_exponent(amax);
+            q[i] = __nv_cvt_float_to_fp8(scalbnf(h[n], -e), __NV_SATFINITE, __NV_E4M3);
+            if (m_local == 0 && n < c.nrows)
+              p.out_sf[static_cast<size_t>(mb) * p.ld_out_sf + c.o_row + n] =
+                  0x01010101u * static_cast<uint32_t>(e + 127);
+          }
+          if (n0 < c.nrows)
+            store_block_16x32(static_cast<uint8_t*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
+                                  (mb * kBM + sub * 32),
+                              p.ld_out, c.nrows - n0, q, staging + sub * 2048, lane);
+        }
+        rbuf ^= 1u;
+      } else {
+#pragma unroll
+        for (int n0 = 0; n0 < 32; n0 += 16) {
+          __nv_bfloat16 yv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(acc[0][n0 + i]);
+          if (n0 < c.nrows)
+            store_block_16x32(static_cast<__nv_bfloat16*>(p.out) +
+                                  static_cast<size_t>(c.o_row + n0) * p.ld_out + (mb * kBM + sub * 32),
+                              p.ld_out, c.nrows - n0, yv,
+                              reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ scale warp
+    // Per stage: lane n < rows copies token n's scale of this K block (fp32, or h's UE8M0
+    // word), lanes 0..kATiles-1 the weight tiles' fp32 block scales, with cp.async; each
+    // lane's completion arrives on the stage's full barrier.
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    const int up_rb = p.up_offset / kBM;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+      const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
+      if (c.nrows <= 0) continue;
+      const int mb = tc.mb;
+      const float* wsc = p.fs_w[c.seg] + static_cast<size_t>(c.group) * p.wsf_rb_per_group * p.k_blocks;
+      for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
+        const bool w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        uint8_t* raw = tiles + stage * C::kStageBytes + C::kATiles * kABytes + C::kBBytes;
+        if (lane < c.nrows) {
+          if (MODE == kFFN2X)
+            cp_async_4(raw + lane * 4, p.tsf[c.seg] + static_cast<size_t>(kb) * p.tsf_ld[c.seg] + c.o_row + lane);
+          else
+            cp_async_4(raw + lane * 4, p.fs_a[c.seg] + static_cast<size_t>(c.b_row + lane) * p.fs_a_ld + kb);
+        }
+        if (lane < C::kATiles) {
+          const int rb = C::kGLU ? (lane ? up_rb + mb : mb) : mb;
+          cp_async_4(raw + 128 + lane * 4, wsc + static_cast<size_t>(rb) * p.k_blocks + kb);
+        }
+        cp_async_mbar_arrive_noinc(&full_bar[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
 // ---------------------------------------------------------------- planner
 // Exclusive block-wide scan (1024 threads, <= 2048 entries) of ceil(sz[order[r]] / rows)
 // over ranks r, into base[0..NG].
@@ -929,8 +1259,53 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int MODE>
+static cudaError_t launch_fs(const GemmLaunch& g, cudaStream_t s) {
+  using C = CfgFS<MODE>;
+  DevParams p;
+  for (int i = 0; i < 2; ++i) p.wmap[i] = g.wmap[i];
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < kTokBoxes; ++j) p.tmap[i][j] = g.tmap[i][j];
+  p.chunks = g.chunks;
+  p.n_chunks = g.n_chunks;
+  p.grp_cp = g.grp_cp;
+  p.n_grp = g.n_grp;
+  p.halves = 0;
+  p.router_T = 0;
+  p.n_mblk = g.n_mblk;
+  p.k_blocks = g.k_blocks;
+  p.k_splits = 1;
+  p.k_per_split = g.k_blocks;
+  p.split_stride = 0;
+  p.w_rows_per_group = g.w_rows_per_group;
+  p.up_offset = g.up_offset;
+  p.m_valid = g.m_valid;
+  p.out = g.out;
+  p.ld_out = g.ld_out;
+  p.status = g.status;
+  p.wsf_rb_per_group = g.wsf_rb_per_group;
+  p.out_sf = g.out_sf;
+  p.ld_out_sf = g.ld_out_sf;
+  for (int i = 0; i < 2; ++i) {
+    p.tsf[i] = g.tsf[i];
+    p.tsf_ld[i] = g.tsf_ld[i];
+    p.tsf_rows[i] = g.tsf_rows[i];
+    p.fs_a[i] = g.fs_a[i];
+    p.fs_w[i] = g.fs_w[i];
+  }
+  p.fs_a_ld = g.fs_a_ld;
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_fs_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::kSmemBytes));
+  if (err != cudaSuccess) return err;
+  grouped_gemm_fs_kernel<MODE><<<g.num_sms, C::kThreads, C::kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   switch (g.mode) {
+    case kFFN1X: return launch_fs<kFFN1X>(g, s);
+    case kFFN2X: return launch_fs<kFFN2X>(g, s);
     case kRouter: return launch_mode<kRouter, kChunkRows>(g, s);
     case kFFN1:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1, kChunkRowsNarrow>(g, s);

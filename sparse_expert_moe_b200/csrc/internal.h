@@ -47,12 +47,12 @@ cudaError_t launch_route(const float* logits, int n_partials, long long partial_
 // when the (token chunk, expert block) tiles alone are fewer -- enough to stream
 // Wr quickly, few enough that summing the partial logits stays cheap (at most 32, the
 // route kernel's limit); every split non-empty.  Host only.
-inline int router_splits(int64_t T, int64_t E, int64_t d) {
+inline int router_splits(int64_t T, int64_t E, int64_t d, int64_t max_splits = 32) {
   const int64_t tiles = ((T + 127) / 128) * ((E + 127) / 128);
   const int64_t kb = d / 64;
   if (tiles == 0) return 1;                 // empty batch: nothing to split
   int64_t s = tiles >= 48 ? 1 : 48 / tiles;
-  if (s > 32) s = 32;
+  if (s > max_splits) s = max_splits;
   if (s > kb) s = kb;
   if (s < 1) s = 1;
   const int64_t per = (kb + s - 1) / s;
@@ -98,9 +98,11 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
 // kFFN2M256 / kFFN2M512: FFN2 (bf16) with 256 / 512 weight rows per tile, as two / four
 // 128-row blocks (M512: decode-sized token tiles only).  kFFN1F4 / kFFN2F4: the FP8 GEMMs
 // with FP4 (MXFP4) weights.  kFFN2F8M256 / kFFN2F4M256: FP8 / FP4 FFN2 with two 128-row
-// weight blocks per tile (decode-sized token tiles).
+// weight blocks per tile (decode-sized token tiles).  kFFN1X / kFFN2X: e4m3 GEMMs with
+// arbitrary fp32 block scales (per-K-block partial sums rescaled in fp32).
 enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5,
-                kFFN2M512 = 6, kFFN1F4 = 7, kFFN2F4 = 8, kFFN2F8M256 = 9, kFFN2F4M256 = 10 };
+                kFFN2M512 = 6, kFFN1F4 = 7, kFFN2F4 = 8, kFFN2F8M256 = 9, kFFN2F4M256 = 10,
+                kFFN1X = 11, kFFN2X = 12 };
 
 struct GemmLaunch {
   int mode;
@@ -137,6 +139,11 @@ struct GemmLaunch {
   const void* gsrc[2];
   const int32_t* gidx[2];
   int g_ld;
+  // fp32-scale modes: token scales fp32 [rows][fs_a_ld] (first GEMM) and weight block
+  // scales fp32 [groups][row blocks][k blocks], per segment
+  const float* fs_a[2];
+  int fs_a_ld;
+  const float* fs_w[2];
   // FP4 modes: E8M0 weight scale codes per segment in 512-byte atoms
   // [groups][rows / 128][K / 128][32 x 16 bytes] (row r, K run q at (r % 32) * 16 + (r / 32) * 4 + q)
   const uint4* wsc[2];
@@ -166,8 +173,9 @@ bool make_tmap_fp4(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
 // x e4m3 [T, d] + x_scale fp32 [T, d/128] -> x_bf16 [T, d] (exact) and x_sf [d/128][T]
 // (UE8M0 replicated x4).  Either output may be null.  Scales that are not positive normal
 // powers of two record MOE_ERR_DEVICE_VALUE in *status (both functions).
+// x_lo (optional): the bf16 remainder v - bf16(v) of each value v = code x scale.
 cudaError_t launch_act_prep_fp8(const uint8_t* x, const float* x_scale, int T, int d, void* x_bf16,
-                                uint32_t* x_sf, int* status, cudaStream_t s);
+                                uint32_t* x_sf, int* status, cudaStream_t s, void* x_lo = nullptr);
 // fp32 power-of-two block scales [n] -> UE8M0 replicated x16 [n] (uint4).
 cudaError_t launch_weight_sf(const float* scales, size_t n, uint4* out, int* status, cudaStream_t s);
 // x_perm_sf[kb][r] = x_sf[kb][perm_token[r]] for r < offsets_total (device).

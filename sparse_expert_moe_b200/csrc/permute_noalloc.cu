@@ -61,7 +61,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   if (cfg->act == MOE_BF16 && (cfg->weight == MOE_E4M3 || cfg->weight == MOE_E2M1))
     return MOE_ERR_UNSUPPORTED;
   // e4m3 rows come with one fp32 scale per 128 channels, permuted alongside the rows
-  const bool fp8 = cfg->act == MOE_E4M3;
+  const bool fp8 = cfg->act == MOE_E4M3 || cfg->act == MOE_E4M3_FP32_SCALE;
   if (fp8 && cfg->T > 0 && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
   const int64_t counts = static_cast<int64_t>(permute_chunks(cfg->T)) * cfg->E;
   if (counts > kMaxCountInts) return MOE_ERR_UNSUPPORTED;   // beyond the fixed scratch

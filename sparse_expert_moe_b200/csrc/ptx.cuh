@@ -285,6 +285,23 @@ __host__ __device__ constexpr uint32_t idesc_mx_bs(int a_fmt, int b_fmt, int M, 
 constexpr int kFmtE4M3 = 0;
 constexpr int kFmtE2M1 = 5;
 
+// Instruction descriptor of kind::f8f6f4 without block scaling: e4m3 A and B (formats 0),
+// fp32 accumulator (bit 4), both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T over K = 32 e4m3 elements, no scale factors.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // e4m3 A and B, scale byte 0 (the FP8 path's scales are replicated across the word).
 __host__ __device__ constexpr uint32_t idesc_e4m3_bs(int M, int N) {
   return idesc_mx_bs(kFmtE4M3, kFmtE4M3, M, N, 0, 0);

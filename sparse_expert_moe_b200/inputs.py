@@ -32,6 +32,8 @@ More, Smaller Experts" -- 384 experts, top-8 plus one shared expert):
                   scale per 32 elements along K)
   r1_decode_fp4q  r1_decode (bf16 activations) with MXFP4 weights: the activations are
                   quantised to e4m3 in the permutation
+  r1_decode_fp8s  r1_decode_fp8 with block scales that are not powers of two (each scale
+                  multiplied by a seeded factor in [1, 2))
 """
 from __future__ import annotations
 
@@ -48,7 +50,7 @@ RECIPE_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file
                           "tests", "golden", "recipes")
 
 # stream ids
-_X, _WR, _BIAS, _W13, _W2, _WS13, _WS2, _XRE, _LOGITS, _ZIPF = range(1, 11)
+_X, _WR, _BIAS, _W13, _W2, _WS13, _WS2, _XRE, _LOGITS, _ZIPF, _FS = range(1, 12)
 _FAMILY = {"tiny": 1, "r1": 2, "kimi": 3, "custom": 9}
 
 W_STD = 0.02
@@ -93,6 +95,8 @@ SPECS = {
                           "e2m1", "bf16", family="r1", x_stream=2, bias_range=0.1),
     "r1_decode_fp4q": Spec("r1_decode_fp4q", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "bf16",
                            "e2m1", "bf16", family="r1", x_stream=2, bias_range=0.1),
+    "r1_decode_fp8s": Spec("r1_decode_fp8s", 128, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3_fs",
+                           "e4m3_fs", "bf16", family="r1", x_stream=2, bias_range=0.1),
     "r1_prefill_fp8": Spec("r1_prefill_fp8", 8192, 7168, 256, 8, 2048, 1, "sigmoid_bias", "e4m3",
                            "e4m3", "bf16", family="r1", x_stream=3, loads="zipf"),
 }
@@ -199,6 +203,17 @@ def redraw_row(spec: Spec, seed: int, t: int, attempt: int) -> np.ndarray:
         spec.d_model, dtype=np.float32)
 
 
+def is_e4m3(dtype: str) -> bool:
+    """e4m3 storage: power-of-two block scales ("e4m3") or any fp32 block scales ("e4m3_fs")."""
+    return dtype in ("e4m3", "e4m3_fs")
+
+
+def _fs_mantissas(shape, *key):
+    """Block-scale multipliers in [1, 2) for the "e4m3_fs" storage: the stored values are the
+    e4m3 codes times (power-of-two scale x multiplier), so no block scale is a power of two."""
+    return _rng(0, _FS, *key).uniform(1.0, 2.0, shape).astype(np.float32)
+
+
 def encode_act(spec: Spec, x32: np.ndarray):
     if spec.act == "f32":
         return torch.from_numpy(np.ascontiguousarray(x32)), None
@@ -206,10 +221,14 @@ def encode_act(spec: Spec, x32: np.ndarray):
         return to_bf16(x32), None
     if spec.act == "e4m3":
         return to_e4m3_blocks(x32, 1, 128)
+    if spec.act == "e4m3_fs":
+        q, s = to_e4m3_blocks(x32, 1, 128)
+        m = _fs_mantissas(s.shape, _FAMILY[spec.family], spec.x_stream, spec.T, spec.d_model)
+        return q, torch.from_numpy(s.numpy() * m)
     raise ValueError(spec.act)
 
 
-def _encode_weight(spec: Spec, w32: np.ndarray):
+def _encode_weight(spec: Spec, w32: np.ndarray, key=()):
     if spec.weight == "f32":
         return torch.from_numpy(np.ascontiguousarray(w32)), None
     if spec.weight == "bf16":
@@ -219,6 +238,9 @@ def _encode_weight(spec: Spec, w32: np.ndarray):
     if spec.weight == "e2m1":
         q, s = to_mxfp4(w32)
         return q, scale_atoms(s.numpy())
+    if spec.weight == "e4m3_fs":
+        q, s = to_e4m3_blocks(w32, 128, 128)
+        return q, torch.from_numpy(s.numpy() * _fs_mantissas(s.shape, _FAMILY[spec.family], *key))
     raise ValueError(spec.weight)
 
 
@@ -232,8 +254,8 @@ def draw_expert(spec: Spec, seed: int, e: int, shared: bool = False):
     r2 = _rng(seed, fam, _WS2 if shared else _W2, e)
     w2 = r2.standard_normal((d, I), dtype=np.float32)
     w2 *= np.float32(W_STD)
-    q13, s13 = _encode_weight(spec, w13)
-    q2, s2 = _encode_weight(spec, w2)
+    q13, s13 = _encode_weight(spec, w13, (int(shared), e, 13))
+    q2, s2 = _encode_weight(spec, w2, (int(shared), e, 2))
     return q13, s13, q2, s2
 
 
@@ -316,10 +338,11 @@ def _stack_experts(spec, seed, n, shared, threads):
         s2 = torch.empty((n, d // 128, I // 128, 512), dtype=torch.uint8)
         scaled = True
     else:
-        wdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[spec.weight]
+        wdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn,
+               "e4m3_fs": torch.float8_e4m3fn}[spec.weight]
         w13 = torch.empty((n, 2 * I, d), dtype=wdt)
         w2 = torch.empty((n, d, I), dtype=wdt)
-        scaled = spec.weight == "e4m3"
+        scaled = is_e4m3(spec.weight)
         s13 = torch.empty((n, 2 * I // 128, d // 128), dtype=torch.float32) if scaled else None
         s2 = torch.empty((n, d // 128, I // 128), dtype=torch.float32) if scaled else None
 

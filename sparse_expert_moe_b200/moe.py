@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_INDEX", 6: "MOE_ERR_TIMEOUT",
                 7: "MOE_ERR_DEVICE_VALUE"}
 SCORE = {"softmax": 0, "sigmoid_bias": 1}
-DTYPE = {"f32": 0, "bf16": 1, "e4m3": 2, "e2m1": 3}
+DTYPE = {"f32": 0, "bf16": 1, "e4m3": 2, "e2m1": 3, "e4m3_fs": 4}
 
 
 class MoeError(RuntimeError):
@@ -252,7 +252,8 @@ def moe_status_string(code: int) -> str:
 # a resident layer: weights and workspace on the device
 # ---------------------------------------------------------------------------
 
-_TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}
+_TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn,
+                "e4m3_fs": torch.float8_e4m3fn}
 
 
 @dataclass

@@ -36,7 +36,7 @@ FIT_ETA = 0.5
 def _values(spec, x32):
     """Real values the layer sees for fp32 activation draws x32 (after storage encoding)."""
     x, xs = inputs.encode_act(spec, x32)
-    if spec.act == "e4m3":
+    if inputs.is_e4m3(spec.act):
         import torch
         return oracle.dequantize_blocks(x.view(torch.uint8).numpy(), xs.numpy(), 1, 128)
     return x.double().numpy()
@@ -119,7 +119,9 @@ def make(name: str, seed: int = 0) -> dict:
         for t in bad:
             attempts[t] += 1
             x32[t] = inputs.redraw_row(spec, seed, int(t), int(attempts[t]))
-        xv_bad = _values(spec, x32[bad])
+        # encode whole matrices: a storage whose block scales carry per-matrix factors
+        # ("e4m3_fs") does not encode a subset of rows the same way
+        xv_bad = _values(spec, x32)[bad]
         gaps = _gaps(spec, _keys(spec, xv_bad, wr, bias64))
         bad = bad[gaps < spec.margin]
     rec["redraw"] = [[int(t), int(a)] for t, a in enumerate(attempts) if a]

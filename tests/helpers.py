@@ -44,7 +44,7 @@ def margin_logits(T, E, k, score, bias, margin=1e-3, seed=0, stream=0):
 
 
 def act_values(wl) -> np.ndarray:
-    if wl.spec.act == "e4m3":
+    if inputs.is_e4m3(wl.spec.act):
         return oracle.dequantize_blocks(wl.x.view(torch.uint8).numpy(), wl.x_scale.numpy(), 1, 128)
     return wl.x.double().numpy()
 
@@ -58,7 +58,7 @@ def margin_workload(spec, seed=0, threads=None):
     while True:
         x32 = inputs._draw_x_fp32(spec, seed, sorted(attempts.items()))
         x, xs = inputs.encode_act(spec, x32)
-        xv = x.double().numpy() if spec.act != "e4m3" else oracle.dequantize_blocks(
+        xv = x.double().numpy() if not inputs.is_e4m3(spec.act) else oracle.dequantize_blocks(
             x.view(torch.uint8).numpy(), xs.numpy(), 1, 128)
         keys = oracle.selection_keys(oracle.router_logits(xv, wr), spec.score, b64)
         bad = np.nonzero(topk_gaps(keys, spec.top_k) < spec.margin)[0]

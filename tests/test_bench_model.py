@@ -54,5 +54,7 @@ def test_launch_count_per_layer_call():
     assert bench.launches_per_step(inputs.SPECS["r1_decode"]) == 8
     assert bench.launches_per_step(inputs.SPECS["r1_prefill"]) == 9
     assert bench.launches_per_step(inputs.SPECS["kimi"]) == 9
-    assert bench.launches_per_step(inputs.SPECS["r1_prefill_fp8"]) == 15
+    assert bench.launches_per_step(inputs.SPECS["r1_prefill_fp8"]) == 13   # rows gathered by FFN1
+    assert bench.launches_per_step(inputs.SPECS["r1_decode_fp8"]) == 14
+    assert bench.launches_per_step(inputs.SPECS["r1_decode_fp4q"]) == 8
     assert bench.launches_per_step(inputs.SPECS["tiny"]) == 12

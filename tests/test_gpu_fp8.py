@@ -201,6 +201,61 @@ def test_quantising_permute_drops_out_of_range_pairs():
     assert np.array_equal(x_perm_s.cpu().numpy()[: R - 2].astype(np.float64), sc[pt])
 
 
+def _e4m3_any_scale(a, br, bc, rng):
+    """e4m3 codes with block scales that are not powers of two: the power-of-two scales of
+    the encoding times factors in [1, 2) (the stored values are codes x these scales)."""
+    q, s = inputs.to_e4m3_blocks(np.asarray(a, np.float32), br, bc)
+    return q, torch.from_numpy(s.numpy() * rng.uniform(1.0, 2.0, s.shape).astype(np.float32))
+
+
+@pytest.mark.parametrize("sizes,d,I", [
+    ([5, 0, 1, 130, 16, 17, 0, 112], 256, 256),
+    ([300], 128, 384),
+    ([1, 2, 3], 512, 128),
+    ([33, 0, 64, 7], 1024, 256),
+])
+def test_grouped_ffn_fp32_block_scales_vs_oracle(sizes, d, I):
+    """e4m3 rows and weights whose block scales are arbitrary fp32 values (MOE_E4M3_FP32_SCALE):
+    every 128-K block rescaled in fp32; h requantised to e4m3 as on the power-of-two path."""
+    rng = np.random.default_rng(sum(sizes) + d + 7)
+    G, n_rows = len(sizes), sum(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    a, a_s = _e4m3_any_scale(rng.standard_normal((n_rows, d)) * np.exp2(rng.integers(-3, 3, (n_rows, 1))),
+                             1, 128, rng)
+    w13 = [_e4m3_any_scale(rng.standard_normal((2 * I, d)) * 0.05 * 2.0 ** rng.integers(-2, 3), 128, 128, rng)
+           for _ in range(G)]
+    w2 = [_e4m3_any_scale(rng.standard_normal((d, I)) * 0.05 * 2.0 ** rng.integers(-2, 3), 128, 128, rng)
+          for _ in range(G)]
+    assert not np.all(np.log2(a_s.numpy()) == np.round(np.log2(a_s.numpy())))
+    cfg = moe.make_config(n_rows, d, G, 1, I, 0, act="e4m3_fs", weight="e4m3_fs")
+    ws = torch.zeros(moe.moe_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    y = torch.full((n_rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_ffn(cfg, G, torch.from_numpy(offsets).to(DEV), n_rows, a.view(torch.uint8).to(DEV),
+                        a_s.to(DEV), torch.stack([q for q, _ in w13]).view(torch.uint8).to(DEV),
+                        torch.stack([s for _, s in w13]).to(DEV),
+                        torch.stack([q for q, _ in w2]).view(torch.uint8).to(DEV),
+                        torch.stack([s for _, s in w2]).to(DEV), y, ws)
+    assert moe.moe_read_device_status(ws) == 0
+    av = _dq(a, a_s, 1, 128)
+    ref = np.zeros((n_rows, d))
+    for g in range(G):
+        lo, hi = offsets[g], offsets[g + 1]
+        if hi > lo:
+            ref[lo:hi] = oracle.swiglu_expert(av[lo:hi], _dq(*w13[g], 128, 128), _dq(*w2[g], 128, 128))
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert max_rel_err(got, ref) < TOL_FP8
+
+
+@pytest.mark.parametrize("T,d,E,k,I,S", [(70, 256, 16, 4, 256, 1), (300, 384, 8, 2, 128, 2),
+                                         (1, 128, 4, 1, 128, 1)])
+def test_layer_fp32_block_scales(T, d, E, k, I, S):
+    spec = inputs.custom_spec(T, d, E, k, I, S, act="e4m3_fs", weight="e4m3_fs")
+    wl = margin_workload(spec, seed=T + 11)
+    assert not np.all(np.log2(wl.w13_s.numpy()) == np.round(np.log2(wl.w13_s.numpy())))
+    _check_fp8_layer(wl)
+
+
 def test_permute_fp8_rows_and_scales():
     T, E, k, d = 300, 32, 4, 256
     rng = np.random.default_rng(9)
@@ -277,7 +332,8 @@ def test_layer_bf16_activations_low_precision_experts(T, d, E, k, I, S, weight):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["r1_decode_fp8", "r1_decode_fp4", "r1_decode_fp4q"])
+@pytest.mark.parametrize("name", ["r1_decode_fp8", "r1_decode_fp4", "r1_decode_fp4q",
+                                  "r1_decode_fp8s"])
 def test_layer_r1_decode_low_precision_full(name):
     """The DeepSeek-R1 decode layer with e4m3 activations and e4m3 or MXFP4 weights, every
     token checked."""

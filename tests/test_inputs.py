@@ -51,7 +51,7 @@ def test_e4m3_scales_are_powers_of_two_and_in_range():
 
 def _routing_of(w):
     spec = w.spec
-    if spec.act == "e4m3":
+    if inputs.is_e4m3(spec.act):
         xv = oracle.dequantize_blocks(w.x.view(torch.uint8).numpy(), w.x_scale.numpy(), 1, 128)
     else:
         xv = w.x.double().numpy()

@@ -209,6 +209,15 @@ def test_table_dequant_helper_equals_oracle():
         assert np.array_equal(a[~np.isnan(a)], b[~np.isnan(b)])
 
 
+def test_block_dequant_takes_any_scale():
+    """A block scale that is not a power of two multiplies each decoded code as it is."""
+    codes = np.full((2, 256), 0x38, np.uint8)           # e4m3 1.0
+    codes[1, 128] = 0xC0                                # e4m3 -2.0
+    s = np.array([[0.3, 1.7], [5.0, 0.1]])
+    v = oracle.dequantize_blocks(codes, s, 1, 128)
+    assert v[0, 0] == 0.3 and v[0, 200] == 1.7 and v[1, 5] == 5.0 and v[1, 128] == -0.2
+
+
 def test_softmax_k_equals_E_is_full_softmax():
     rng = np.random.default_rng(0)
     L = rng.uniform(-3, 3, (32, 7))
