@@ -780,12 +780,16 @@ struct CfgFS {
   static constexpr uint32_t kStageBytes = kATiles * kABytes + kBBytes + kRawBytes;
   static constexpr int kStages = (192u * 1024u) / kStageBytes > 10 ? 10 : (192u * 1024u) / kStageBytes;
   static constexpr uint32_t kPCols = kATiles * kNT;               // per partial buffer
-  static constexpr uint32_t kTmemCols = 2 * kPCols <= 64 ? 64 : 128;
+  // partial buffers in flight: each K block's round trip (MMAs, commit, the epilogue's
+  // TMEM loads and release) spans several K blocks of the weight stream
+  static constexpr int kPBufs = 4;
+  static constexpr uint32_t kTmemCols =
+      kPBufs * kPCols <= 64 ? 64 : (kPBufs * kPCols <= 128 ? 128 : 256);
   static constexpr int kThreads = 224;
   static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;
   static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t kRedBytes = 2 * 4 * 128 * 4;
-  static constexpr uint32_t kPScaleBytes = 2 * 64 * 4;            // [2 buffers][32 token + 2 weight]
+  static constexpr uint32_t kPScaleBytes = kPBufs * 64 * 4;       // [buffers][32 token + 2 weight]
   static constexpr uint32_t kFixedBytes =
       1024 + kStagingBytes + kGrpBytes + kRedBytes + kPScaleBytes + 1024;
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kFixedBytes;
@@ -803,9 +807,9 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
   uint8_t* tiles = smem;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
   uint64_t* empty_bar = full_bar + C::kStages;
-  uint64_t* pfull = empty_bar + C::kStages;                      // [2] partial buffer written
-  uint64_t* pempty = pfull + 2;                                  // [2] partial buffer read
-  uint64_t* red_bar = pempty + 2;                                // [2] amax exchange
+  uint64_t* pfull = empty_bar + C::kStages;                      // [kPBufs] partial buffer written
+  uint64_t* pempty = pfull + C::kPBufs;                          // [kPBufs] partial buffer read
+  uint64_t* red_bar = pempty + C::kPBufs;                        // [2] amax exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* staging = smem + C::kStages * C::kStageBytes + 1024;
@@ -820,11 +824,11 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
       mbar_init(&full_bar[i], 1 + 32);
       mbar_init(&empty_bar[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kPBufs; ++i) {
       mbar_init(&pfull[i], 2);        // the MMAs' commit + the scales' copy
       mbar_init(&pempty[i], 4);       // one arrival per epilogue warp
-      mbar_init(&red_bar[i], 4);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&red_bar[i], 4);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.wmap[0]);
@@ -885,41 +889,43 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t kc = 0;                 // K blocks issued so far (partial buffer kc % 2)
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
-        const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
-        if (c.nrows <= 0) continue;
-        const int n_pad = (c.nrows + 15) & ~15;
-        const uint32_t idesc = idesc_e4m3_f32(kBM, n_pad);
-        for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++kc) {
-          const uint32_t b = kc & 1u;
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.status) ||
-              !mbar_wait(&pempty[b], ((kc >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
+    // The whole warp waits; lane n moves token n's scale, lane 0 issues the MMAs.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t kc = 0;                   // K blocks issued so far (partial buffer kc % kPBufs)
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
+      const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
+      if (c.nrows <= 0) continue;
+      const int n_pad = (c.nrows + 15) & ~15;
+      const uint32_t idesc = idesc_e4m3_f32(kBM, n_pad);
+      for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++kc) {
+        const uint32_t b = kc % C::kPBufs;
+        const bool w = mbar_wait(&full_bar[stage], phase, abort_flag, p.status) &&
+                       mbar_wait(&pempty[b], ((kc / C::kPBufs) & 1u) ^ 1u, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* st = tiles + stage * C::kStageBytes;
+        const uint8_t* raw = st + C::kATiles * kABytes + C::kBBytes;
+        float* ps = pscale + b * 64;
+        // this K block's scales to the buffer's slot: token n's (fp32, or h's UE8M0 word
+        // -> 2^(code - 127)) and each weight tile's fp32 block scale
+        if (lane < c.nrows) {
+          if (MODE == kFFN2X) {
+            const uint32_t code = reinterpret_cast<const uint32_t*>(raw)[lane] & 0xFFu;
+            ps[lane] = code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
+          } else {
+            ps[lane] = reinterpret_cast<const float*>(raw)[lane];
           }
-          tc_fence_after();
+        }
+        if (lane < C::kATiles) ps[32 + lane] = reinterpret_cast<const float*>(raw + 128)[lane];
+        __syncwarp();
+        if (lane == 0) {
           fence_proxy_async_smem();    // the scale warp's cp.async rows before any async read
-          const uint8_t* st = tiles + stage * C::kStageBytes;
-          const uint8_t* raw = st + C::kATiles * kABytes + C::kBBytes;
-          float* ps = pscale + b * 64;
-          // this K block's scales to the buffer's slot: token n's (fp32, or h's UE8M0 word
-          // -> 2^(code - 127)) and each weight tile's fp32 block scale
-          for (int n = 0; n < c.nrows; ++n) {
-            if (MODE == kFFN2X) {
-              const uint32_t code = reinterpret_cast<const uint32_t*>(raw)[n] & 0xFFu;
-              ps[n] = code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
-            } else {
-              ps[n] = reinterpret_cast<const float*>(raw)[n];
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < C::kATiles; ++j) ps[32 + j] = reinterpret_cast<const float*>(raw + 128)[j];
           const uint32_t sa = smem_u32(st), sb = sa + C::kATiles * kABytes;
           const uint32_t d0 = tmem_base + b * C::kPCols;
 #pragma unroll
@@ -933,10 +939,11 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
           umma_commit(&empty_bar[stage]);   // the stage's operands and raw scales are consumed
           umma_commit(&pfull[b]);           // the partial sums are in TMEM
           mbar_arrive(&pfull[b]);           // the scales are in their slot
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
     }
@@ -958,8 +965,8 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
 #pragma unroll
         for (int n = 0; n < 32; ++n) acc[j][n] = 0.f;
       for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++kc) {
-        const uint32_t b = kc & 1u;
-        const bool w = mbar_wait(&pfull[b], (kc >> 1) & 1u, abort_flag, p.status);
+        const uint32_t b = kc % C::kPBufs;
+        const bool w = mbar_wait(&pfull[b], (kc / C::kPBufs) & 1u, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
