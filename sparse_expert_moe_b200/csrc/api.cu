@@ -394,7 +394,9 @@ moe_status run_ffn_fs(const moe_config& c, const Layout& L, void* ws, const FsSe
   if (st != MOE_OK) return st;
   if (ev && (st = cuda_status(cudaEventRecord(ev[0], s))) != MOE_OK) return st;
 
-  g.mode = kFFN2X;
+  // two 128-row weight blocks (256 output columns) per tile, as d_model allows
+  const bool m256 = d % 256 == 0;
+  g.mode = m256 ? kFFN2XM256 : kFFN2X;
   if (!make_tok_maps(g.tmap[0], h, rows_all, I, true)) return MOE_ERR_CUDA;
   copy_maps(g.tmap[1], g.tmap[0]);
   for (int i = 0; i < 2; ++i) {
@@ -405,7 +407,7 @@ moe_status run_ffn_fs(const moe_config& c, const Layout& L, void* ws, const FsSe
     g.tsf_ld[i] = static_cast<int>(rows_all);
     g.tsf_rows[i] = static_cast<int>(rows_all);
   }
-  g.n_mblk = static_cast<int>(d / 128);
+  g.n_mblk = static_cast<int>(m256 ? d / 256 : d / 128);
   g.k_blocks = static_cast<int>(I / 128);
   g.w_rows_per_group = static_cast<int>(d);
   g.wsf_rb_per_group = static_cast<int>(d / 128);

@@ -88,8 +88,8 @@ struct DevParams {
   const uint8_t* gsrc[2];
   const int32_t* gidx[2];
   int g_ld;
-  // fp32-scale modes (kFFN1X / kFFN2X): token scales fp32 [rows][fs_a_ld] per segment
-  // (kFFN1X; kFFN2X reads h's UE8M0 words through tsf), weight scales fp32
+  // fp32-scale modes (kFFN1X / kFFN2X / kFFN2XM256): token scales fp32 [rows][fs_a_ld] per
+  // segment (kFFN1X; the second GEMM reads h's UE8M0 words through tsf), weight scales fp32
   // [groups][row blocks][k blocks] per segment
   const float* fs_a[2];
   int fs_a_ld;
@@ -773,7 +773,10 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW, GATHER>::kThreads, 1)
 template <int MODE>
 struct CfgFS {
   static constexpr bool kGLU = MODE == kFFN1X;
-  static constexpr int kATiles = kGLU ? 2 : 1;
+  static constexpr bool kSecond = MODE == kFFN2X || MODE == kFFN2XM256;   // reads h
+  // FFN2: 128-row weight blocks (= 128 output columns each) per tile
+  static constexpr int kOutBlocks = MODE == kFFN2XM256 ? 2 : 1;
+  static constexpr int kATiles = kGLU ? 2 : kOutBlocks;
   static constexpr int kNT = kChunkRowsNarrow;                    // 32 tokens
   static constexpr uint32_t kBBytes = kNT * kRowBytes;
   static constexpr uint32_t kRawBytes = 1024;                     // [32] token + [2] weight scales
@@ -782,9 +785,11 @@ struct CfgFS {
   static constexpr uint32_t kPCols = kATiles * kNT;               // per partial buffer
   // partial buffers in flight: each K block's round trip (MMAs, commit, the epilogue's
   // TMEM loads and release) spans several K blocks of the weight stream
-  static constexpr int kPBufs = 4;
+  static constexpr int kPBufs = 8;
   static constexpr uint32_t kTmemCols =
-      kPBufs * kPCols <= 64 ? 64 : (kPBufs * kPCols <= 128 ? 128 : 256);
+      kPBufs * kPCols <= 64 ? 64
+                            : (kPBufs * kPCols <= 128 ? 128 : (kPBufs * kPCols <= 256 ? 256 : 512));
+  static_assert(kPBufs * kPCols <= 512, "TMEM budget");
   static constexpr int kThreads = 224;
   static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;
   static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;
@@ -856,9 +861,9 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
         const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
         const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
         if (c.nrows <= 0) continue;
-        const int a_row = c.group * p.w_rows_per_group + tc.mb * kBM;
+        const int a_row = c.group * p.w_rows_per_group + tc.mb * kBM * C::kOutBlocks;
         const int n_pad = (c.nrows + 15) & ~15;
-        const int tok_row = MODE == kFFN2X ? c.o_row : c.b_row;
+        const int tok_row = C::kSecond ? c.o_row : c.b_row;
         const uint32_t bytes = C::kATiles * kABytes + n_pad * kRowBytes;
         const CUtensorMap* wm = &p.wmap[c.seg];
         for (int kb = tc.kb0; kb < tc.kb1; ++kb) {
@@ -871,6 +876,9 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           tma_load_2d(st, wm, &full_bar[stage], kx, a_row);
           if (C::kGLU) tma_load_2d(st + kABytes, wm, &full_bar[stage], kx, a_row + p.up_offset);
+#pragma unroll
+          for (int j = 1; j < C::kOutBlocks; ++j)
+            tma_load_2d(st + j * kABytes, wm, &full_bar[stage], kx, a_row + j * kBM);
           uint8_t* bt = st + C::kATiles * kABytes;
           for (int bi = 0, off = 0; bi < kTokBoxes; ++bi) {
             const int rows = 128 >> bi;
@@ -915,7 +923,7 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
         // this K block's scales to the buffer's slot: token n's (fp32, or h's UE8M0 word
         // -> 2^(code - 127)) and each weight tile's fp32 block scale
         if (lane < c.nrows) {
-          if (MODE == kFFN2X) {
+          if (C::kSecond) {
             const uint32_t code = reinterpret_cast<const uint32_t*>(raw)[lane] & 0xFFu;
             ps[lane] = code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
           } else {
@@ -1027,16 +1035,20 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
         }
         rbuf ^= 1u;
       } else {
+        // accumulator j holds output columns (mb * kOutBlocks + j) * 128 + (0..127)
 #pragma unroll
-        for (int n0 = 0; n0 < 32; n0 += 16) {
-          __nv_bfloat16 yv[16];
+        for (int j = 0; j < C::kATiles; ++j) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(acc[0][n0 + i]);
-          if (n0 < c.nrows)
-            store_block_16x32(static_cast<__nv_bfloat16*>(p.out) +
-                                  static_cast<size_t>(c.o_row + n0) * p.ld_out + (mb * kBM + sub * 32),
-                              p.ld_out, c.nrows - n0, yv,
-                              reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+          for (int n0 = 0; n0 < 32; n0 += 16) {
+            __nv_bfloat16 yv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(acc[j][n0 + i]);
+            if (n0 < c.nrows)
+              store_block_16x32(static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
+                                    ((mb * C::kOutBlocks + j) * kBM + sub * 32),
+                                p.ld_out, c.nrows - n0, yv,
+                                reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+          }
         }
       }
     }
@@ -1063,13 +1075,13 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
         }
         uint8_t* raw = tiles + stage * C::kStageBytes + C::kATiles * kABytes + C::kBBytes;
         if (lane < c.nrows) {
-          if (MODE == kFFN2X)
+          if (C::kSecond)
             cp_async_4(raw + lane * 4, p.tsf[c.seg] + static_cast<size_t>(kb) * p.tsf_ld[c.seg] + c.o_row + lane);
           else
             cp_async_4(raw + lane * 4, p.fs_a[c.seg] + static_cast<size_t>(c.b_row + lane) * p.fs_a_ld + kb);
         }
         if (lane < C::kATiles) {
-          const int rb = C::kGLU ? (lane ? up_rb + mb : mb) : mb;
+          const int rb = C::kGLU ? (lane ? up_rb + mb : mb) : mb * C::kOutBlocks + lane;
           cp_async_4(raw + 128 + lane * 4, wsc + static_cast<size_t>(rb) * p.k_blocks + kb);
         }
         cp_async_mbar_arrive_noinc(&full_bar[stage]);
@@ -1313,6 +1325,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   switch (g.mode) {
     case kFFN1X: return launch_fs<kFFN1X>(g, s);
     case kFFN2X: return launch_fs<kFFN2X>(g, s);
+    case kFFN2XM256: return launch_fs<kFFN2XM256>(g, s);
     case kRouter: return launch_mode<kRouter, kChunkRows>(g, s);
     case kFFN1:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1, kChunkRowsNarrow>(g, s);

@@ -102,7 +102,7 @@ cudaError_t launch_plan(const int32_t* offsets, int G, int n_rows, int n_shared,
 // arbitrary fp32 block scales (per-K-block partial sums rescaled in fp32).
 enum GemmMode { kRouter = 0, kFFN1 = 1, kFFN2 = 2, kFFN1F8 = 3, kFFN2F8 = 4, kFFN2M256 = 5,
                 kFFN2M512 = 6, kFFN1F4 = 7, kFFN2F4 = 8, kFFN2F8M256 = 9, kFFN2F4M256 = 10,
-                kFFN1X = 11, kFFN2X = 12 };
+                kFFN1X = 11, kFFN2X = 12, kFFN2XM256 = 13 };
 
 struct GemmLaunch {
   int mode;
