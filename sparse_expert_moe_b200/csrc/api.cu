@@ -135,6 +135,12 @@ int bf16_chunk_rows(int64_t max_group) {
   return max_group <= kChunkRows ? kChunkRowsNarrow : kChunkRowsWide;
 }
 
+// fp32-scale chunk rows: 32 for decode-sized batches, else 64 (the token tiles of the
+// fp32-scale GEMMs, whose accumulators live in registers).
+int fs_chunk_rows(int64_t max_group) {
+  return max_group <= kChunkRows ? kChunkRowsNarrow : 2 * kChunkRowsNarrow;
+}
+
 // FP8 / FP4-weight chunk rows: 32 for decode-sized batches (groups of at most 128 rows:
 // small token tiles leave shared memory to the weight stream), else 112, or 224 once
 // groups can exceed 112 rows (FFN2 tiles of 224 tokens, FFN1 tiles of half a chunk).
@@ -356,7 +362,7 @@ struct FsSeg {
 };
 
 moe_status run_ffn_fs(const moe_config& c, const Layout& L, void* ws, const FsSeg& s0,
-                      const FsSeg& s1, int64_t rows_all, void* y, cudaStream_t s,
+                      const FsSeg& s1, int64_t rows_all, void* y, int chunk_rows, cudaStream_t s,
                       cudaEvent_t* ev = nullptr) {
   const int64_t d = c.d_model, I = c.d_ff;
   void* h = at<void>(ws, L.h);
@@ -371,6 +377,7 @@ moe_status run_ffn_fs(const moe_config& c, const Layout& L, void* ws, const FsSe
   g.num_sms = num_sms();
 
   g.mode = kFFN1X;
+  g.tile_tokens = chunk_rows;        // one chunk per tile: 32 or 64 tokens
   for (int i = 0; i < 2; ++i) {
     const FsSeg& q = *seg[i];
     if (!make_tmap_u8(&g.wmap[i], q.w13, q.groups * 2 * I, d, 128) ||
@@ -590,14 +597,15 @@ moe_status moe_grouped_ffn(const moe_config* cfg, int32_t n_groups, const int32_
   }
   if (fp32_scaled(*cfg)) {   // e4m3 rows and weights with arbitrary fp32 block scales
     if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
-    st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, kChunkRowsNarrow,
+    const int chunk_rows = fs_chunk_rows(n_rows);
+    st = cuda_status(launch_plan(group_offsets, n_groups, n_rows, 0, cfg->T, 0, chunk_rows,
                                  at<Chunk>(ws, L.chunks), at<int32_t>(ws, kHdrNChunks * sizeof(int)),
                                  at<int32_t>(ws, L.grp_cp), at<int32_t>(ws, kHdrNGroups * sizeof(int)),
                                  status_word(ws), stream));
     if (st != MOE_OK) return st;
     const FsSeg s0{a, a_scale, n_rows, w13, w2, static_cast<const float*>(w13_s),
                    static_cast<const float*>(w2_s), n_groups};
-    return run_ffn_fs(*cfg, L, ws, s0, FsSeg{}, n_rows, y, stream);
+    return run_ffn_fs(*cfg, L, ws, s0, FsSeg{}, n_rows, y, chunk_rows, stream);
   }
   if (tok_e4m3(*cfg)) {   // e4m3 token rows (as moe_permute gives them for e4m3 / FP4 experts)
     if (!a_scale || !w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
@@ -797,8 +805,9 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
   // here; otherwise the rows are copied into x_perm (bf16 rows, or e4m3 rows + scale
   // factors).  bf16 rows keep the copy: measured on the R1 prefill layer, the first GEMM
   // fed by TMA from x_perm is faster than with gathered rows by more than the copy costs.
-  const int chunk_rows = fs ? kChunkRowsNarrow : (fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T));
-  const bool gather = fp8 && chunk_rows != kChunkRowsNarrow;
+  const int chunk_rows = fs ? fs_chunk_rows(T) : (fp8 ? fp8_chunk_rows(T) : bf16_chunk_rows(T));
+  // (the fp32-scale GEMMs read their token rows from x_perm at every width)
+  const bool gather = fp8 && !fs && chunk_rows != kChunkRowsNarrow;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm_token = at<int32_t>(ws, L.perm_token);
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
@@ -849,7 +858,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* wts, con
                    static_cast<const float*>(wts->w13_s), static_cast<const float*>(wts->w2_s), E};
     const FsSeg s1{x_b, x_scale, T, ws13_b, ws2_b, static_cast<const float*>(wts->ws13_s),
                    static_cast<const float*>(wts->ws2_s), S};
-    st = run_ffn_fs(c, L, ws, s0, s1, L.rows_all, y_rows, s, ev ? ev + 5 : nullptr);
+    st = run_ffn_fs(c, L, ws, s0, s1, L.rows_all, y_rows, chunk_rows, s, ev ? ev + 5 : nullptr);
   } else if (fp8) {
     Fp8Seg s0{x_perm, x_perm_sf, R, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E, nullptr};
     if (gather) s0 = Fp8Seg{x_tok, x_sf, T, w13_b, w2_b, nullptr, nullptr, nullptr, nullptr, E, perm_token};

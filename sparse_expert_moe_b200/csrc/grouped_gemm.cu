@@ -762,39 +762,46 @@ __global__ void __launch_bounds__(Cfg<MODE, NTW, GATHER>::kThreads, 1)
 // e4m3 expert GEMMs whose block scales are arbitrary positive fp32 values (not powers of
 // two, which the tensor cores' UE8M0 scale factors cannot hold).  The MMAs run without
 // block scaling (kind::f8f6f4); every 128-K block accumulates into its own TMEM buffer
-// (two, alternating), and the epilogue warps fold it into fp32 register accumulators as
+// (several in rotation), and the epilogue warps fold it into fp32 register accumulators as
 //   acc[r][n] += (s_w[block of r][kb] * s_a[n][kb]) * partial_kb[r][n]
 // -- the block-scaled product summed exactly as its definition states, in fp32.  Tiles are
-// 32 tokens wide (the accumulators of a tile live in registers), 128 weight rows (two
-// tiles, gate and up, for the first GEMM).
+// NT = 32 tokens wide on decode-sized batches, else 64 (the accumulators of a tile live in
+// registers: each epilogue warp holds 32 tokens of its 32 weight rows, so a 64-token tile
+// has two sets of four epilogue warps), and 128 weight rows per weight tile (gate and up
+// for the first GEMM; one or two output blocks for the second).
 //   warp 0  TMA producer; warp 1  MMA issuer (also moves each block's scales from the stage
-//   to a per-buffer slot the epilogue reads); warps 2-5  epilogue; warp 6  scale warp
-//   (cp.async of the stage's raw token and weight scales).
-template <int MODE>
+//   to a per-buffer slot the epilogue reads); warps 2 .. 2 + 4 NT / 32 - 1  epilogue; the
+//   last warp  scale warp (cp.async of the stage's raw token and weight scales).
+template <int MODE, int NT>
 struct CfgFS {
   static constexpr bool kGLU = MODE == kFFN1X;
   static constexpr bool kSecond = MODE == kFFN2X || MODE == kFFN2XM256;   // reads h
   // FFN2: 128-row weight blocks (= 128 output columns each) per tile
   static constexpr int kOutBlocks = MODE == kFFN2XM256 ? 2 : 1;
   static constexpr int kATiles = kGLU ? 2 : kOutBlocks;
-  static constexpr int kNT = kChunkRowsNarrow;                    // 32 tokens
+  static constexpr int kNT = NT;                                  // 32 or 64 tokens
+  static_assert(NT == 32 || NT == 64, "token tile width");
+  static constexpr int kEpiWarps = 4 * (kNT / 32);                // four per 32 tokens
+  static constexpr int kScaleWarp = 2 + kEpiWarps;
   static constexpr uint32_t kBBytes = kNT * kRowBytes;
-  static constexpr uint32_t kRawBytes = 1024;                     // [32] token + [2] weight scales
+  static constexpr uint32_t kRawBytes = 1024;                     // [kNT] token + [2] weight scales
+  static constexpr uint32_t kRawW = kNT * 4;                      // weight scales in the raw block
   static constexpr uint32_t kStageBytes = kATiles * kABytes + kBBytes + kRawBytes;
   static constexpr int kStages = (192u * 1024u) / kStageBytes > 10 ? 10 : (192u * 1024u) / kStageBytes;
   static constexpr uint32_t kPCols = kATiles * kNT;               // per partial buffer
   // partial buffers in flight: each K block's round trip (MMAs, commit, the epilogue's
   // TMEM loads and release) spans several K blocks of the weight stream
-  static constexpr int kPBufs = 8;
+  static constexpr int kPBufs = 512 / kPCols < 8 ? 512 / kPCols : 8;
   static constexpr uint32_t kTmemCols =
       kPBufs * kPCols <= 64 ? 64
                             : (kPBufs * kPCols <= 128 ? 128 : (kPBufs * kPCols <= 256 ? 256 : 512));
   static_assert(kPBufs * kPCols <= 512, "TMEM budget");
-  static constexpr int kThreads = 224;
-  static constexpr uint32_t kStagingBytes = 4 * 16 * 32 * 4;
-  static constexpr uint32_t kGrpBytes = 2 * (kMaxGroups + 1) * 4;
-  static constexpr uint32_t kRedBytes = 2 * 4 * 128 * 4;
-  static constexpr uint32_t kPScaleBytes = kPBufs * 64 * 4;       // [buffers][32 token + 2 weight]
+  static constexpr int kThreads = 32 * (3 + kEpiWarps);
+  static constexpr uint32_t kStagingBytes = kEpiWarps * 16 * 32 * 4;
+  static constexpr uint32_t kGrpBytes = (2 * (kMaxGroups + 1) * 4 + 15) & ~15u;   // 16-byte multiple
+  static constexpr uint32_t kRedBytes = 2 * 4 * kNT * 4;          // [2][4 row quadrants][kNT]
+  static constexpr int kSlot = kNT + 32;                          // floats per scale slot
+  static constexpr uint32_t kPScaleBytes = kPBufs * kSlot * 4;    // [buffers][kNT token + 2 weight]
   static constexpr uint32_t kFixedBytes =
       1024 + kStagingBytes + kGrpBytes + kRedBytes + kPScaleBytes + 1024;
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kFixedBytes;
@@ -802,10 +809,10 @@ struct CfgFS {
   static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
 };
 
-template <int MODE>
-__global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
+template <int MODE, int NT>
+__global__ void __launch_bounds__(CfgFS<MODE, NT>::kThreads, 1)
     grouped_gemm_fs_kernel(const __grid_constant__ DevParams p) {
-  using C = CfgFS<MODE>;
+  using C = CfgFS<MODE, NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -831,9 +838,9 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
     }
     for (int i = 0; i < C::kPBufs; ++i) {
       mbar_init(&pfull[i], 2);        // the MMAs' commit + the scales' copy
-      mbar_init(&pempty[i], 4);       // one arrival per epilogue warp
+      mbar_init(&pempty[i], C::kEpiWarps);   // one arrival per epilogue warp
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&red_bar[i], 4);
+    for (int i = 0; i < 2; ++i) mbar_init(&red_bar[i], C::kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.wmap[0]);
@@ -919,18 +926,20 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
         tc_fence_after();
         const uint8_t* st = tiles + stage * C::kStageBytes;
         const uint8_t* raw = st + C::kATiles * kABytes + C::kBBytes;
-        float* ps = pscale + b * 64;
+        float* ps = pscale + b * C::kSlot;
         // this K block's scales to the buffer's slot: token n's (fp32, or h's UE8M0 word
         // -> 2^(code - 127)) and each weight tile's fp32 block scale
-        if (lane < c.nrows) {
+#pragma unroll
+        for (int n = lane; n < C::kNT; n += 32) {
+          if (n >= c.nrows) break;
           if (C::kSecond) {
-            const uint32_t code = reinterpret_cast<const uint32_t*>(raw)[lane] & 0xFFu;
-            ps[lane] = code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
+            const uint32_t code = reinterpret_cast<const uint32_t*>(raw)[n] & 0xFFu;
+            ps[n] = code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
           } else {
-            ps[lane] = reinterpret_cast<const float*>(raw)[lane];
+            ps[n] = reinterpret_cast<const float*>(raw)[n];
           }
         }
-        if (lane < C::kATiles) ps[32 + lane] = reinterpret_cast<const float*>(raw + 128)[lane];
+        if (lane < C::kATiles) ps[C::kNT + lane] = reinterpret_cast<const float*>(raw + C::kRawW)[lane];
         __syncwarp();
         if (lane == 0) {
           fence_proxy_async_smem();    // the scale warp's cp.async rows before any async read
@@ -956,10 +965,14 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < C::kScaleWarp) {
     // ------------------------------------------------------------ epilogue
+    // Warp 2 + e: TMEM lane quadrant warp % 4 (32 weight rows), tokens 32 (e / 4) .. + 31.
     const int sub = warp & 3;
+    const int e_warp = warp - 2;
+    const int n_base = C::kNT > 32 ? (e_warp >> 2) * 32 : 0;   // this warp's first token
     const int m_local = sub * 32 + lane;      // weight row inside the tile
+    uint8_t* stg = staging + e_warp * 2048;
     uint32_t kc = 0;
     uint32_t rbuf = 0, rpar = 0;
     bool ok = true;
@@ -967,6 +980,7 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
       const TileCoord tc = tile_coord(p, t, grp_cp, n_grp);
       const Chunk c = tile_rows<MODE, kChunkRowsNarrow>(p, tc);
       if (c.nrows <= 0) continue;
+      const int rows = c.nrows - n_base;      // this warp's tokens (<= 0: none; warp-uniform)
       float acc[C::kATiles][32];
 #pragma unroll
       for (int j = 0; j < C::kATiles; ++j)
@@ -980,17 +994,20 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const float* ps = pscale + b * 64;
-        const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::kPCols;
+        if (rows > 0) {
+          const float* ps = pscale + b * C::kSlot;
+          const uint32_t tb =
+              tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::kPCols + n_base;
 #pragma unroll
-        for (int j = 0; j < C::kATiles; ++j) {
-          float v0[16], v1[16];
-          tmem_ld16x2(tb + j * C::kNT, tb + j * C::kNT + 16, v0, v1);
-          const float sw = ps[32 + j];
+          for (int j = 0; j < C::kATiles; ++j) {
+            float v0[16], v1[16];
+            tmem_ld16x2(tb + j * C::kNT, tb + j * C::kNT + 16, v0, v1);
+            const float sw = ps[C::kNT + j];
 #pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            acc[j][n] = fmaf(sw * ps[n], v0[n], acc[j][n]);
-            acc[j][16 + n] = fmaf(sw * ps[16 + n], v1[n], acc[j][16 + n]);
+            for (int n = 0; n < 16; ++n) {
+              acc[j][n] = fmaf(sw * ps[n_base + n], v0[n], acc[j][n]);
+              acc[j][16 + n] = fmaf(sw * ps[n_base + 16 + n], v1[n], acc[j][16 + n]);
+            }
           }
         }
         tc_fence_before();
@@ -999,16 +1016,19 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
       }
       if (!ok) break;
       const int mb = tc.mb;
+      const int o_row = c.o_row + n_base;     // this warp's first output row
       if (MODE == kFFN1X) {
         // SwiGLU, then h requantised to e4m3 with one power-of-two scale per token per 128 h
-        // columns, exchanged between the four epilogue warps (as the block-scaled path does)
+        // columns, exchanged between the four warps of the token's rows (as the block-scaled
+        // path does); every epilogue warp arrives on the exchange barrier
+        constexpr int kRR = C::kNT;
         float h[32];
-        uint32_t* redt = red + rbuf * (4 * 128);
+        uint32_t* redt = red + rbuf * (4 * kRR);
 #pragma unroll
         for (int n = 0; n < 32; ++n) {
           h[n] = acc[0][n] / (1.0f + __expf(-acc[0][n])) * acc[1][n];
           const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h[n])));
-          if (lane == 0) redt[sub * 128 + n] = wmax;
+          if (lane == 0) redt[sub * kRR + n_base + n] = wmax;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_bar[rbuf]);
@@ -1020,18 +1040,19 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
           uint8_t q[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int n = n0 + i;
-            const uint32_t amax = max(max(redt[n], redt[128 + n]), max(redt[256 + n], redt[384 + n]));
+            const int n = n_base + n0 + i;
+            const uint32_t amax =
+                max(max(redt[n], redt[kRR + n]), max(redt[2 * kRR + n], redt[3 * kRR + n]));
             const int e = e4m3_scale_exponent(amax);
-            q[i] = __nv_cvt_float_to_fp8(scalbnf(h[n], -e), __NV_SATFINITE, __NV_E4M3);
-            if (m_local == 0 && n < c.nrows)
-              p.out_sf[static_cast<size_t>(mb) * p.ld_out_sf + c.o_row + n] =
+            q[i] = __nv_cvt_float_to_fp8(scalbnf(h[n0 + i], -e), __NV_SATFINITE, __NV_E4M3);
+            if (m_local == 0 && n0 + i < rows)
+              p.out_sf[static_cast<size_t>(mb) * p.ld_out_sf + o_row + n0 + i] =
                   0x01010101u * static_cast<uint32_t>(e + 127);
           }
-          if (n0 < c.nrows)
-            store_block_16x32(static_cast<uint8_t*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
+          if (n0 < rows)
+            store_block_16x32(static_cast<uint8_t*>(p.out) + static_cast<size_t>(o_row + n0) * p.ld_out +
                                   (mb * kBM + sub * 32),
-                              p.ld_out, c.nrows - n0, q, staging + sub * 2048, lane);
+                              p.ld_out, rows - n0, q, stg, lane);
         }
         rbuf ^= 1u;
       } else {
@@ -1043,20 +1064,19 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
             __nv_bfloat16 yv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) yv[i] = __float2bfloat16_rn(acc[j][n0 + i]);
-            if (n0 < c.nrows)
-              store_block_16x32(static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(c.o_row + n0) * p.ld_out +
+            if (n0 < rows)
+              store_block_16x32(static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(o_row + n0) * p.ld_out +
                                     ((mb * C::kOutBlocks + j) * kBM + sub * 32),
-                                p.ld_out, c.nrows - n0, yv,
-                                reinterpret_cast<__nv_bfloat16*>(staging + sub * 2048), lane);
+                                p.ld_out, rows - n0, yv, reinterpret_cast<__nv_bfloat16*>(stg), lane);
           }
         }
       }
     }
   } else {
     // ------------------------------------------------------------ scale warp
-    // Per stage: lane n < rows copies token n's scale of this K block (fp32, or h's UE8M0
-    // word), lanes 0..kATiles-1 the weight tiles' fp32 block scales, with cp.async; each
-    // lane's completion arrives on the stage's full barrier.
+    // Per stage: lanes copy the tile's token scales of this K block (token n by lane n % 32;
+    // fp32, or h's UE8M0 word), lanes 0..kATiles-1 the weight tiles' fp32 block scales, with
+    // cp.async; each lane's completion arrives on the stage's full barrier.
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -1074,15 +1094,17 @@ __global__ void __launch_bounds__(CfgFS<MODE>::kThreads, 1)
           break;
         }
         uint8_t* raw = tiles + stage * C::kStageBytes + C::kATiles * kABytes + C::kBBytes;
-        if (lane < c.nrows) {
+#pragma unroll
+        for (int n = lane; n < C::kNT; n += 32) {
+          if (n >= c.nrows) break;
           if (C::kSecond)
-            cp_async_4(raw + lane * 4, p.tsf[c.seg] + static_cast<size_t>(kb) * p.tsf_ld[c.seg] + c.o_row + lane);
+            cp_async_4(raw + n * 4, p.tsf[c.seg] + static_cast<size_t>(kb) * p.tsf_ld[c.seg] + c.o_row + n);
           else
-            cp_async_4(raw + lane * 4, p.fs_a[c.seg] + static_cast<size_t>(c.b_row + lane) * p.fs_a_ld + kb);
+            cp_async_4(raw + n * 4, p.fs_a[c.seg] + static_cast<size_t>(c.b_row + n) * p.fs_a_ld + kb);
         }
         if (lane < C::kATiles) {
           const int rb = C::kGLU ? (lane ? up_rb + mb : mb) : mb * C::kOutBlocks + lane;
-          cp_async_4(raw + 128 + lane * 4, wsc + static_cast<size_t>(rb) * p.k_blocks + kb);
+          cp_async_4(raw + C::kRawW + lane * 4, wsc + static_cast<size_t>(rb) * p.k_blocks + kb);
         }
         cp_async_mbar_arrive_noinc(&full_bar[stage]);
         if (++stage == C::kStages) {
@@ -1278,9 +1300,9 @@ static cudaError_t launch_mode(const GemmLaunch& g, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int MODE>
+template <int MODE, int NT>
 static cudaError_t launch_fs(const GemmLaunch& g, cudaStream_t s) {
-  using C = CfgFS<MODE>;
+  using C = CfgFS<MODE, NT>;
   DevParams p;
   for (int i = 0; i < 2; ++i) p.wmap[i] = g.wmap[i];
   for (int i = 0; i < 2; ++i)
@@ -1313,19 +1335,26 @@ static cudaError_t launch_fs(const GemmLaunch& g, cudaStream_t s) {
     p.fs_w[i] = g.fs_w[i];
   }
   p.fs_a_ld = g.fs_a_ld;
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_fs_kernel<MODE>,
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_fs_kernel<MODE, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::kSmemBytes));
   if (err != cudaSuccess) return err;
-  grouped_gemm_fs_kernel<MODE><<<g.num_sms, C::kThreads, C::kSmemBytes, s>>>(p);
+  grouped_gemm_fs_kernel<MODE, NT><<<g.num_sms, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   switch (g.mode) {
-    case kFFN1X: return launch_fs<kFFN1X>(g, s);
-    case kFFN2X: return launch_fs<kFFN2X>(g, s);
-    case kFFN2XM256: return launch_fs<kFFN2XM256>(g, s);
+    // fp32-scale GEMMs: 32-token tiles on decode-sized batches, else 64
+    case kFFN1X:
+      return g.tile_tokens == 2 * kChunkRowsNarrow ? launch_fs<kFFN1X, 2 * kChunkRowsNarrow>(g, s)
+                                                   : launch_fs<kFFN1X, kChunkRowsNarrow>(g, s);
+    case kFFN2X:
+      return g.tile_tokens == 2 * kChunkRowsNarrow ? launch_fs<kFFN2X, 2 * kChunkRowsNarrow>(g, s)
+                                                   : launch_fs<kFFN2X, kChunkRowsNarrow>(g, s);
+    case kFFN2XM256:
+      return g.tile_tokens == 2 * kChunkRowsNarrow ? launch_fs<kFFN2XM256, 2 * kChunkRowsNarrow>(g, s)
+                                                   : launch_fs<kFFN2XM256, kChunkRowsNarrow>(g, s);
     case kRouter: return launch_mode<kRouter, kChunkRows>(g, s);
     case kFFN1:
       if (g.tile_tokens == kChunkRowsNarrow) return launch_mode<kFFN1, kChunkRowsNarrow>(g, s);
