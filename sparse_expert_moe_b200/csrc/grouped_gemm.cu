@@ -789,8 +789,9 @@ struct CfgFS {
   static constexpr uint32_t kStageBytes = kATiles * kABytes + kBBytes + kRawBytes;
   static constexpr int kStages = (192u * 1024u) / kStageBytes > 10 ? 10 : (192u * 1024u) / kStageBytes;
   static constexpr uint32_t kPCols = kATiles * kNT;               // per partial buffer
-  // partial buffers in flight: each K block's round trip (MMAs, commit, the epilogue's
-  // TMEM loads and release) spans several K blocks of the weight stream
+  // partial buffers in flight (eight, or as many as TMEM holds): each K block's round trip
+  // (MMAs, commit, the epilogue's TMEM loads and release) spans several K blocks of the
+  // weight stream
   static constexpr int kPBufs = 512 / kPCols < 8 ? 512 / kPCols : 8;
   static constexpr uint32_t kTmemCols =
       kPBufs * kPCols <= 64 ? 64
