@@ -102,7 +102,8 @@ typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_BIAS = 1 } moe_score_fn;
  * for weights, as for MOE_E4M3) may be any positive finite value, not only powers of two.
  * The expert GEMMs then multiply without block scaling and fold each 128-K block's
  * s_weight * s_activation into fp32 accumulators (exact up to fp32 rounding), on 32-token
- * tiles: slower than MOE_E4M3, whose power-of-two scales the tensor cores apply directly.
+ * tiles for decode-sized batches and 64-token tiles above: slower than MOE_E4M3, whose
+ * power-of-two scales the tensor cores apply directly.
  * Activations and weights both take this dtype.  The router takes x = code x scale as a
  * bf16 part plus its bf16 remainder (two router GEMMs, summed with the split-K partials):
  * x to ~2^-17 relative, where a single bf16 rounding would move the logits by ~2^-9. */
