@@ -43,6 +43,21 @@ def test_workspace_size_host_only(lib):
     assert moe.moe_workspace_size(tiny) > 0
 
 
+def test_low_precision_workspaces_host_only(lib):
+    """Every accepted low-precision family sizes its workspace without a GPU, decode- and
+    prefill-sized (the fp32-scale family keeps x_perm and its fp32 scales at every width)."""
+    for T in (128, 8192):
+        for act, weight in (("e4m3", "e4m3"), ("e4m3", "e2m1"), ("bf16", "e4m3"), ("bf16", "e2m1"),
+                            ("e4m3_fs", "e4m3_fs")):
+            cfg = moe.make_config(T, 7168, 256, 8, 2048, 1, act=act, weight=weight)
+            n = moe.moe_workspace_size(cfg)
+            # at least h (e4m3) and the bf16 expert outputs: (T*k + T) * (I + 2 d)
+            assert n >= T * 9 * (2048 + 2 * 7168), (T, act, weight)
+            if act == "e4m3_fs":
+                # plus x_perm (e4m3) and its fp32 1x128 scales
+                assert n >= T * 9 * (2048 + 2 * 7168) + T * 8 * 7168 * (1 + 4 / 128)
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(top_k=9, E=8), 2),                    # k > E
     (dict(top_k=17, E=64), 2),                  # k > 16
@@ -51,6 +66,10 @@ def test_workspace_size_host_only(lib):
     (dict(d_ff=200), 2),                        # I % 128
     (dict(T=-1), 1),                            # negative size
     (dict(act="e4m3", weight="bf16"), 2),       # mixed dtype family
+    (dict(act="e4m3_fs", weight="e4m3"), 2),    # fp32-scale rows need fp32-scale weights
+    (dict(act="e4m3", weight="e4m3_fs"), 2),    # ... and the converse
+    (dict(act="bf16", weight="e4m3_fs"), 2),    # no quantising permutation to fp32 scales
+    (dict(act="e2m1", weight="e2m1"), 2),       # FP4 is a weight format only
 ])
 def test_config_rejections(lib, kw, code):
     base = dict(T=16, d_model=256, E=8, top_k=2, d_ff=256, n_shared=1)
